@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Indexer throughput on B200: query-key pairs scored and selected per second.
+
+A step is one pass of the whole hot path over the decode-batch workload
+(32 sequences x 32768 cached keys, H_I=64, d_I=128, bf16, top_k=2048, one query per
+sequence): append the step's new keys to the cache, score every (query, key) pair
+(tensor-core logits + fused ReLU / head-weighted sum), select the top 2048 per
+query.  Steps are captured in a CUDA graph and replayed; the K cache (268 MB) is
+larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank processes its own 32 sequences (weak scaling, no
+collective on the data path); the time is the max over ranks and `value` counts
+the pairs of all ranks.  `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "indexer query-key pairs scored+selected/sec (prefill & decode); % of roofline"
+UNIT = "pairs/s"
+WORKLOAD = "decode batch: 32 seqs x 32768 keys, H_I=64, d_I=128, bf16, top_k=2048, 1 query/seq"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--graph-steps", type=int, default=50, help="steps captured per CUDA graph")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work for the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- workload
+
+def workload(rank: int):
+    from sparse_attention_token_02_b200 import workloads as W
+    return W.decode(seed=2 + 1000 * rank)
+
+
+def host_inputs(wl):
+    from sparse_attention_token_02_b200 import workloads as W
+    return W.make_inputs(wl)
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def _oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _oracle_row(wl, inp, b, n_keys):
+    """One decode row of sequence b restricted to its first n_keys keys, through the oracle."""
+    import oracle
+    kv = oracle.bf16_bits_to_f64(inp["k_bits"][b][:n_keys])
+    qv = oracle.bf16_bits_to_f64(inp["q_bits"][b: b + 1])
+    res = oracle.decode_oracle(qv, [kv], inp["w"][b: b + 1].astype(np.float64), [n_keys], 1, wl.top_k)
+    assert res["idx"].shape == (1, wl.top_k)
+    return n_keys
+
+
+def oracle_sample(wl, inp, seconds: float):
+    """Times the fp64 oracle on whole decode rows of this workload until `seconds` pass."""
+    pairs = rows = b = 0
+    t0 = time.perf_counter()
+    while True:
+        pairs += _oracle_row(wl, inp, b, wl.seq_lens[b])
+        rows += 1
+        b = (b + 1) % wl.num_seqs
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": pairs / dt, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"{rows} whole decode rows of {wl.seq_lens[0]} keys (numpy fp64 oracle, {dt:.1f} s)"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is a bounded sample of the workload
+    (whole rows when the step budget allows, else a row's first keys, at least top_k+1),
+    sized so that warm-up plus all steps take about two and a half minutes."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = workload(0)
+    inp = host_inputs(wl)
+    L = wl.seq_lens[0]
+    t = time.perf_counter()
+    _oracle_row(wl, inp, 0, L)
+    row_s = time.perf_counter() - t
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    if budget >= row_s:
+        rows_per_step, keys = max(1, min(wl.num_seqs, int(budget / row_s))), L
+    else:
+        rows_per_step, keys = 1, int(min(L, max(wl.top_k + 1, L * budget / row_s)))
+    secs, pairs = [], 0
+    b = 0
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        n = 0
+        for _ in range(rows_per_step):
+            n += _oracle_row(wl, inp, b, keys)
+            b = (b + 1) % wl.num_seqs
+        if i >= args.warmup:
+            secs.append(time.perf_counter() - t)
+            pairs += n
+    value = pairs / sum(secs)
+    sample = (f"per step {rows_per_step} decode row(s) x {keys} keys of the workload "
+              f"(numpy fp64 oracle; {len(secs)} steps, {sum(secs):.1f} s)")
+    info = {"value": value, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle", "sample": sample}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": info,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str | None):
+        self.lines = []
+        self.proc = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if device_uuid:
+            cmd += ["-i", device_uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self, t_begin: float, t_end: float):
+        """Summary of the samples taken between the wall-clock times t_begin and t_end."""
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        import datetime
+        sm, mx, reasons, n_all = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, mx = float(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            n_all += 1
+            if not (t_begin - 0.1 <= ts <= t_end + 0.1):
+                continue
+            sm.append(clk)
+            for n, v in zip(names, parts[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0, "samples_total": n_all}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our path
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the decode logits kernel from the committed ncu summary,
+    or None when the kernel source changed since those counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "logits_decode_bf16_traffic.md")
+    src = os.path.join(ROOT, "sparse_attention_token_02_b200", "csrc", "kernels_logits.cu")
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        fields = dict(ln.split(":", 1) for ln in text.splitlines() if ":" in ln and not ln.startswith("#"))
+        if fields.get("kernels_logits_sha256", "").strip() != sha:
+            return None
+        return float(fields["dram_bytes_per_launch"].strip())
+    except Exception:
+        return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_attention_token_02_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream(device=dev)
+
+    wl = workload(rank)
+    inp = host_inputs(wl)
+    S, L, H, d, k = wl.num_seqs, wl.seq_lens[0], wl.H, wl.d, wl.top_k
+    k_base = np.arange(S, dtype=np.int64) * L
+    seq_lens, q_lens = [L] * S, [1] * S
+
+    with torch.cuda.stream(stream):
+        cache = api.IndexerKCache.empty(S * L, d, fp8=False, device=dev)
+        k_all = torch.from_numpy(np.concatenate(inp["k_bits"]).view(np.int16)).view(torch.bfloat16).to(dev)
+        api.dsa_indexer_kcache_append(cache, k_all, torch.arange(S * L, dtype=torch.int64, device=dev), stream=stream)
+        del k_all
+        q = torch.from_numpy(inp["q_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+        w = torch.from_numpy(inp["w"]).to(dev)
+        # the step's new key of each sequence: its last cache row (re-appended every step)
+        k_new_bits = np.stack([kb[-1] for kb in inp["k_bits"]])
+        k_new = torch.from_numpy(k_new_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        dst_rows = torch.from_numpy(k_base + L - 1).to(dev)
+        out_idx = torch.empty(S, k, dtype=torch.int32, device=dev)
+        out_score = torch.empty(S, k, dtype=torch.float32, device=dev)
+    stream.synchronize()
+
+    def step():
+        api.dsa_indexer_kcache_append(cache, k_new, dst_rows, stream=stream)
+        api.dsa_indexer_decode(q, cache, w, seq_lens, q_lens, k, k_base=k_base, out_idx=out_idx,
+                               out_score=out_score, stream=stream)
+
+    # uncaptured warm-up (also plans the batch once)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    api.dsa_check_device_errors(stream)
+
+    # capture G steps, each with its own kernel-timing events
+    G = max(1, min(args.graph_steps, args.steps))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(G)]
+    with torch.cuda.stream(stream):
+        for trio in ev:
+            for e in trio:
+                e.record(stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    n0 = api.dsa_kernel_launch_count()
+    with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
+        for g in range(G):
+            api.dsa_set_profile_events(*ev[g])
+            step()
+        api.dsa_set_profile_events(None, None, None)
+    launches_per_step = (api.dsa_kernel_launch_count() - n0) / G
+    replays = max(1, args.steps // G)
+    K = replays * G
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            graph.replay()
+    stream.synchronize()
+    api.dsa_check_device_errors(stream)
+
+    # timed region
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    time.sleep(0.5)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(replays):
+            graph.replay()
+        t1.record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop(wall0, wall1)
+    ms_total = t0.elapsed_time(t1)
+    logits_ms = statistics.mean(ev[g][0].elapsed_time(ev[g][1]) for g in range(G))
+    topk_ms = statistics.mean(ev[g][1].elapsed_time(ev[g][2]) for g in range(G))
+    api.dsa_check_device_errors(stream)
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / K
+    pairs_step = wl.pairs * world
+    value = pairs_step / (ms_step * 1e-3)
+
+    # end to end through the host-buffer entry point: upload inputs, run, read results back
+    q_h = torch.from_numpy(inp["q_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    w_h = torch.from_numpy(inp["w"]).pin_memory()
+    k_h = torch.from_numpy(k_new_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    rows_h = torch.from_numpy(k_base + L - 1).pin_memory()
+    bufs = {}
+    for _ in range(5):
+        api.dsa_indexer_decode_from_host(q_h, w_h, k_h, rows_h, cache, seq_lens, q_lens, k, k_base=k_base,
+                                         dev_bufs=bufs, stream=stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    E = max(1, args.e2e_steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(E):
+        api.dsa_indexer_decode_from_host(q_h, w_h, k_h, rows_h, cache, seq_lens, q_lens, k, k_base=k_base,
+                                         dev_bufs=bufs, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / E
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, w_h, k_h, rows_h))
+    d2h = S * k * (4 + 4)
+
+    # roofline of the dominant kernel (decode logits): algorithmic bytes it must read
+    alg_bytes = S * L * d * 2 + S * H * d * 2 + S * H * 4
+    achieved = alg_bytes / (logits_ms * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    traffic = profiled_traffic()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(wl, inp, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "pairs_per_step_per_gpu": wl.pairs,
+                       "l2": "inputs larger than L2 (268 MB bf16 K cache per GPU), no flush",
+                       "step": "kcache_append + decode (logits + top-k), CUDA graph of %d steps" % G,
+                       "parallelism": f"{world} independent ranks (sequences sharded)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "logits (decode, bf16)", "kernel_ms": logits_ms,
+                         "peak_source": f"{peak_kind} hbm_gbs", "alg_bytes_per_launch": alg_bytes},
+            "kernels_ms": {"logits": logits_ms, "topk": topk_ms},
+            "cpu_baseline": cpu,
+            "e2e": {"value": pairs_step / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": int(round(launches_per_step * K)),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,207 @@
+/*
+ * dsa_indexer.h -- C ABI of the DeepSeek Sparse Attention Lightning Indexer on B200.
+ *
+ * The operation (page "从原理到代码：手把手教你理解DeepSeek-V3.2的闪电索引器设计" §2.1 and §3;
+ * page "Lightning Indexer 详解" §2 and §4; page "Study MLA Indexer", section 数学流):
+ *
+ *     I[t, s] = sum_{i < H_I} w[t, i] * ReLU( q[t, i, :] . k[s, :] / sqrt(d_I) )
+ *
+ * for every query t and every cached key s at or before t's position, with ONE
+ * d_I-dimensional indexer key per token shared by all H_I heads; then the
+ * top_k largest I[t, s] per query (DeepSeek-V3.2 uses top_k = 2048).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named "device" are CUDA device pointers on the current device;
+ *   "host" pointers are read synchronously during the call and may be reused
+ *   as soon as it returns.  Device pointers passed to the tensor-core path (the
+ *   cache, the queries) must be 16-byte aligned.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *   only enqueues work on it; outputs are valid once the stream has reached
+ *   that point.  Calls that share a stream may be issued back to back.
+ * - Ownership: the library never frees or keeps caller memory.  It owns a
+ *   workspace per (device, stream), grown on demand with cudaMalloc, unless
+ *   the caller supplies one with dsa_set_workspace().
+ * - Errors: argument problems are found before anything is enqueued and
+ *   returned as a status; dsa_get_last_error() then holds a message (per
+ *   thread).  Faults detected inside kernels (a cache row out of range, a
+ *   bounded wait that expired, a broken selection invariant) are recorded in
+ *   a device flag and reported by dsa_check_device_errors().
+ * - Positions: the keys of a step are appended BEFORE scoring ("Study MLA
+ *   Indexer", 两条 cache 区分), so a sequence with seq_len keys and q_len
+ *   queries has its query j at position p = seq_len - q_len + j and that
+ *   query sees keys 0..p (itself included).
+ * - Output: for query row r, out_idx[r*top_k + j] (int32) are 0-based key
+ *   positions inside the query's sequence and out_score[r*top_k + j] (fp32)
+ *   their scores.  The min(top_k, p+1) valid entries come first; the rest are
+ *   -1 / -inf.  The order of the valid entries is unspecified: the result is
+ *   the index SET of "Lightning Indexer 详解" §1.  Among keys whose scores are
+ *   exactly equal at the k-th place, which ones are kept is unspecified.
+ */
+#ifndef DSA_INDEXER_H
+#define DSA_INDEXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_INDEXER_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+typedef enum {
+  DSA_BF16 = 0,      /* bfloat16 */
+  DSA_FP8_E4M3 = 1,  /* OCP FP8 E4M3 ("e4m3fn") with one fp32 scale per row */
+  DSA_F32 = 2        /* fp32, accepted as an append / quantise SOURCE only */
+} dsa_dtype_t;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent batch, misalignment */
+  DSA_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for (H_I, d_I, dtype) */
+  DSA_ERR_ALLOC = 3,         /* the library could not allocate its workspace */
+  DSA_ERR_CUDA = 4,          /* a CUDA runtime call failed (message has the CUDA error) */
+  DSA_ERR_DEVICE_CHECK = 5   /* a kernel recorded a fault (see dsa_check_device_errors) */
+} dsa_status_t;
+
+/* One layer's indexer key cache, packed by rows.  Sequences live at arbitrary
+ * row ranges (see dsa_batch_t.k_base).  Row r holds the key of one token. */
+typedef struct {
+  void* k;                /* device [capacity_rows, d_I] bf16 or e4m3 bytes, row-major        */
+  float* k_scale;         /* device [capacity_rows] fp32 per-row scale (FP8), NULL for bf16    */
+  int64_t capacity_rows;  /* rows allocated in k (and k_scale)                                */
+  int32_t d_I;            /* key width: 128 (DeepSeek-V3.2) or 64                              */
+  dsa_dtype_t dtype;      /* DSA_BF16 or DSA_FP8_E4M3                                          */
+} dsa_kcache_t;
+
+/* Queries of all sequences, packed in sequence order: sequence b owns q_lens[b]
+ * consecutive rows. */
+typedef struct {
+  const void* data;       /* device [T_total, H_I, d_I] bf16 or e4m3 bytes                     */
+  const float* scale;     /* device [T_total] fp32 per-token scale (FP8), NULL for bf16        */
+  dsa_dtype_t dtype;      /* must equal the cache dtype                                        */
+  int32_t H_I;            /* indexer heads (64 in DeepSeek-V3.2)                               */
+  int32_t d_I;            /* must equal the cache d_I                                          */
+} dsa_query_t;
+
+/* The ragged batch, described on the host. */
+typedef struct {
+  int32_t num_seqs;
+  const int32_t* seq_lens;  /* host [num_seqs]: cached keys of each sequence, this step's included */
+  const int32_t* q_lens;    /* host [num_seqs]: queries of each sequence; NULL means q_len == seq_len */
+  const int64_t* k_base;    /* host [num_seqs]: cache row holding key position 0 of each sequence;
+                               NULL means the sequences are packed back to back from row 0           */
+} dsa_batch_t;
+
+/*
+ * Append keys to the cache ("Lightning Indexer 详解" §2.1 and §2.4: each new token's
+ * key becomes the next cache row, history is never recomputed; "Study MLA
+ * Indexer", 数学流: the K path is quantised to FP8 before the write).
+ *   k_new     device [n, d_I] source rows, dtype src_dtype (DSA_BF16 or DSA_F32)
+ *   dst_rows  device int64 [n]: destination cache row of each source row
+ * bf16 cache: a copy (fp32 sources rounded to nearest even).  FP8 cache: each row
+ * is quantised with its own scale = absmax / 448 (IEEE fp32 division), codes =
+ * E4M3(x / scale) rounded to nearest even and saturated to +-448; an all-zero
+ * row gets scale 1.  A destination outside [0, capacity_rows) is skipped and
+ * recorded as a device fault.
+ */
+DSA_API dsa_status_t dsa_indexer_kcache_append(const dsa_kcache_t* kc, const void* k_new, dsa_dtype_t src_dtype,
+                                       const int64_t* dst_rows, int32_t n, void* stream);
+
+/*
+ * Per-row FP8 quantisation, the routine the cache append uses; it also
+ * quantises queries with one scale per token over all H_I * d_I values
+ * (row_len = H_I * d_I).
+ *   src    device [rows, row_len] DSA_BF16 or DSA_F32
+ *   dst    device uint8 [rows, row_len] E4M3 codes
+ *   scale  device fp32 [rows]
+ * row_len must be a positive multiple of 16.
+ */
+DSA_API dsa_status_t dsa_quantize_rows_fp8(const void* src, dsa_dtype_t src_dtype, int64_t rows, int32_t row_len,
+                                   uint8_t* dst, float* scale, void* stream);
+
+/*
+ * Prefill: score every query of every sequence against its causal history and
+ * select the top_k keys ("从原理到代码…" §3: scores for all query/key pairs, causal
+ * mask, topk; "Study MLA Indexer", 数学流: [L, L] logits then arg top-k [L, k]).
+ *   q, kc     queries and cache as above (same dtype, same d_I)
+ *   w         device fp32 [T_total, H_I] head weights (any sign; softmax output in
+ *             DeepSeek-V3.2, "从原理到代码…" §2.1)
+ *   batch     host description; T_total = sum(q_lens)
+ *   top_k     >= 1
+ *   out_idx   device int32 [T_total, top_k]
+ *   out_score device fp32  [T_total, top_k]
+ * Supported shapes: (H_I, d_I) = (64, 128) in bf16 or FP8, (4, 64) in bf16.
+ */
+DSA_API dsa_status_t dsa_indexer_prefill(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                 const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx, float* out_score,
+                                 void* stream);
+
+/*
+ * Decode: the same scoring and selection for a step of 1 to 4 new queries per
+ * sequence at the end of each cache ("Lightning Indexer 详解" §2: one query scores
+ * every cached position, linear in L per step).  Arguments as for prefill;
+ * every q_lens[b] must be in 1..4 (q_lens may not be NULL).  The key range of
+ * each sequence is split across the GPU so few long sequences still fill it.
+ * Supported shapes: (H_I, d_I) = (64, 128) in bf16 or FP8.
+ */
+DSA_API dsa_status_t dsa_indexer_decode(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx, float* out_score,
+                                void* stream);
+
+/*
+ * The scores alone, without selection (the first page's index_scores, §3):
+ * out_scores[r * ld + s] = I[p_r, s] for s = 0..p_r.  Entries with s > p_r are
+ * not written.  ld >= max(seq_lens) and ld % 4 == 0.
+ */
+DSA_API dsa_status_t dsa_indexer_scores(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                const dsa_batch_t* batch, float* out_scores, int64_t ld, void* stream);
+
+/* Workspace bytes a call with this batch needs (scores plus scheduling tables). */
+DSA_API size_t dsa_indexer_workspace_bytes(const dsa_query_t* q, const dsa_batch_t* batch, int32_t top_k);
+
+/*
+ * Use caller memory (device, 256-byte aligned) as the workspace of `stream` on
+ * the current device instead of library allocations; ptr == NULL returns to
+ * library-owned memory.  A call whose workspace does not fit returns
+ * DSA_ERR_ALLOC.  The memory must stay valid while work using it is pending.
+ */
+DSA_API dsa_status_t dsa_set_workspace(void* ptr, size_t bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears any device fault recorded by
+ * this library's kernels on that stream: DSA_OK or DSA_ERR_DEVICE_CHECK (the
+ * message names the fault).
+ */
+DSA_API dsa_status_t dsa_check_device_errors(void* stream);
+
+/*
+ * Profiling hook.  Registers three cudaEvent_t for the calling thread (NULL
+ * clears them): every later prefill / decode / scores call on this thread
+ * records ev_begin right before its logits kernel, ev_mid right after it and
+ * ev_end after its last kernel, all on the call's stream.  Timing one step's
+ * kernels this way needs no profiler.
+ */
+DSA_API dsa_status_t dsa_set_profile_events(void* ev_begin, void* ev_mid, void* ev_end);
+
+/* Number of kernels this library has launched from the calling thread so far. */
+DSA_API uint64_t dsa_kernel_launch_count(void);
+
+/* Message of the last failed call on this thread ("" if none). */
+DSA_API const char* dsa_get_last_error(void);
+
+/* Library version string. */
+DSA_API const char* dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_INDEXER_H */

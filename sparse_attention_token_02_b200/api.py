@@ -1,0 +1,234 @@
+"""Python binding of the indexer's C ABI: torch tensors in, pointers out.
+
+Argument marshalling only.  torch provides device memory and the current CUDA
+stream; every step of the indexer runs in the CUDA library.  Names follow the C
+entry points (include/dsa_indexer.h).
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import DSA_BF16, DSA_F32, DSA_FP8_E4M3, Batch, KCache, Query, check
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DSA_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return DSA_FP8_E4M3
+    if t.dtype == torch.float32:
+        return DSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("device tensors must be contiguous CUDA tensors")
+
+
+@dataclass
+class IndexerKCache:
+    """An indexer key cache: ``k`` [capacity, d_I] bf16 or uint8 (E4M3 codes), ``k_scale`` [capacity] fp32 (FP8)."""
+    k: torch.Tensor
+    k_scale: torch.Tensor | None = None
+
+    @staticmethod
+    def empty(capacity: int, d_I: int, fp8: bool, device="cuda") -> "IndexerKCache":
+        if fp8:
+            return IndexerKCache(torch.zeros(capacity, d_I, dtype=torch.uint8, device=device),
+                                 torch.ones(capacity, dtype=torch.float32, device=device))
+        return IndexerKCache(torch.zeros(capacity, d_I, dtype=torch.bfloat16, device=device), None)
+
+    @property
+    def fp8(self) -> bool:
+        return self.k.dtype in (torch.uint8, torch.float8_e4m3fn)
+
+    def c(self) -> KCache:
+        _require_cuda(self.k, self.k_scale)
+        return KCache(self.k.data_ptr(), self.k_scale.data_ptr() if self.k_scale is not None else None,
+                      self.k.shape[0], self.k.shape[1], DSA_FP8_E4M3 if self.fp8 else DSA_BF16)
+
+
+def _query(q: torch.Tensor, q_scale) -> Query:
+    _require_cuda(q, q_scale)
+    if q.dim() != 3:
+        raise ValueError("q must be [T_total, H_I, d_I]")
+    code = _dtype_code(q)
+    return Query(q.data_ptr(), q_scale.data_ptr() if q_scale is not None else None, code, q.shape[1], q.shape[2])
+
+
+class _HostBatch:
+    """Keeps the host arrays of a dsa_batch_t alive for the duration of a call."""
+
+    def __init__(self, seq_lens, q_lens, k_base):
+        self.seq = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+        self.ql = None if q_lens is None else np.ascontiguousarray(np.asarray(q_lens, dtype=np.int32))
+        self.kb = None if k_base is None else np.ascontiguousarray(np.asarray(k_base, dtype=np.int64))
+        self.c = Batch(len(self.seq), self.seq.ctypes.data,
+                       None if self.ql is None else self.ql.ctypes.data,
+                       None if self.kb is None else self.kb.ctypes.data)
+
+    @property
+    def total_q(self) -> int:
+        return int(self.seq.sum() if self.ql is None else self.ql.sum())
+
+
+def dsa_indexer_kcache_append(cache: IndexerKCache, k_new: torch.Tensor, dst_rows: torch.Tensor, stream=None):
+    """Write (bf16 cache) or quantise and write (FP8 cache) rows ``k_new`` [n, d_I] to ``dst_rows`` (int64)."""
+    _require_cuda(k_new, dst_rows)
+    if dst_rows.dtype != torch.int64:
+        raise TypeError("dst_rows must be int64")
+    kc = cache.c()
+    check(_lib.load().dsa_indexer_kcache_append(ctypes.byref(kc), _ptr(k_new), _dtype_code(k_new), _ptr(dst_rows),
+                                                k_new.shape[0], _stream(stream)))
+
+
+def dsa_quantize_rows_fp8(src: torch.Tensor, stream=None):
+    """Per-row FP8 E4M3 quantisation of ``src`` [rows, ...] (bf16 / fp32): returns (codes uint8, scale fp32 [rows])."""
+    _require_cuda(src)
+    rows = src.shape[0]
+    row_len = src.numel() // max(rows, 1) if rows else 0
+    dst = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    scale = torch.empty(rows, dtype=torch.float32, device=src.device)
+    check(_lib.load().dsa_quantize_rows_fp8(_ptr(src), _dtype_code(src), rows, row_len, _ptr(dst), _ptr(scale),
+                                            _stream(stream)))
+    return dst, scale
+
+
+def _run(fn_name, q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score, stream):
+    b = _HostBatch(seq_lens, q_lens, k_base)
+    T = b.total_q
+    _require_cuda(w)
+    if w.dtype != torch.float32:
+        raise TypeError("w must be fp32")
+    if out_idx is None:
+        out_idx = torch.empty(T, top_k, dtype=torch.int32, device=q.device)
+    if out_score is None:
+        out_score = torch.empty(T, top_k, dtype=torch.float32, device=q.device)
+    _require_cuda(out_idx, out_score)
+    qq, kc = _query(q, q_scale), cache.c()
+    fn = getattr(_lib.load(), fn_name)
+    check(fn(ctypes.byref(qq), ctypes.byref(kc), _ptr(w), ctypes.byref(b.c), top_k, _ptr(out_idx), _ptr(out_score),
+             _stream(stream)))
+    return out_idx, out_score
+
+
+def dsa_indexer_prefill(q, cache: IndexerKCache, w, seq_lens, top_k, q_scale=None, q_lens=None, k_base=None,
+                        out_idx=None, out_score=None, stream=None):
+    """Scores + top-k for every query of a ragged batch; returns (out_idx int32, out_score fp32) [T_total, top_k]."""
+    return _run("dsa_indexer_prefill", q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score,
+                stream)
+
+
+def dsa_indexer_decode(q, cache: IndexerKCache, w, seq_lens, q_lens, top_k, q_scale=None, k_base=None,
+                       out_idx=None, out_score=None, stream=None):
+    """A decode step (1..4 queries per sequence at the end of each cache); returns (out_idx, out_score)."""
+    return _run("dsa_indexer_decode", q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score,
+                stream)
+
+
+def dsa_indexer_scores(q, cache: IndexerKCache, w, seq_lens, q_scale=None, q_lens=None, k_base=None, ld=None,
+                       out=None, stream=None):
+    """Dense scores [T_total, ld] (entries after each query's position are left as they were: -inf here)."""
+    b = _HostBatch(seq_lens, q_lens, k_base)
+    if ld is None:
+        ld = (int(b.seq.max()) + 3) // 4 * 4 if len(b.seq) else 4
+    if out is None:
+        out = torch.full((b.total_q, ld), float("-inf"), dtype=torch.float32, device=q.device)
+    _require_cuda(w, out)
+    qq, kc = _query(q, q_scale), cache.c()
+    check(_lib.load().dsa_indexer_scores(ctypes.byref(qq), ctypes.byref(kc), _ptr(w), ctypes.byref(b.c), _ptr(out),
+                                         ld, _stream(stream)))
+    return out
+
+
+def dsa_indexer_workspace_bytes(q, seq_lens, top_k, q_lens=None) -> int:
+    b = _HostBatch(seq_lens, q_lens, None)
+    qq = Query(0, None, _dtype_code(q), q.shape[1], q.shape[2])
+    return int(_lib.load().dsa_indexer_workspace_bytes(ctypes.byref(qq), ctypes.byref(b.c), top_k))
+
+
+def dsa_set_workspace(buf: torch.Tensor | None, stream=None):
+    if buf is None:
+        check(_lib.load().dsa_set_workspace(None, 0, _stream(stream)))
+    else:
+        _require_cuda(buf)
+        check(_lib.load().dsa_set_workspace(_ptr(buf), buf.numel() * buf.element_size(), _stream(stream)))
+
+
+def dsa_check_device_errors(stream=None):
+    """Synchronise the stream and raise if one of the library's kernels recorded a fault."""
+    check(_lib.load().dsa_check_device_errors(_stream(stream)))
+
+
+def dsa_set_profile_events(begin=None, mid=None, end=None):
+    """Register torch.cuda.Event objects (timing enabled) recorded around the next calls' kernels."""
+    v = [None if e is None else ctypes.c_void_p(e.cuda_event) for e in (begin, mid, end)]
+    check(_lib.load().dsa_set_profile_events(*v))
+
+
+def dsa_kernel_launch_count() -> int:
+    return int(_lib.load().dsa_kernel_launch_count())
+
+
+def dsa_version() -> str:
+    return _lib.load().dsa_version().decode()
+
+
+def dsa_indexer_decode_from_host(q_host, w_host, k_new_host, dst_rows, cache: IndexerKCache, seq_lens, q_lens,
+                                 top_k, q_scale_host=None, k_base=None, dev_bufs=None, stream=None):
+    """A whole decode step from pinned HOST buffers: upload the step's new keys, queries
+    and weights, append the keys, score + select, and copy the result back.
+
+    Returns host (out_idx, out_score).  ``dev_bufs`` (a dict) caches device staging
+    tensors between calls.  The copies are enqueued on the same stream as the kernels.
+    """
+    s = torch.cuda.current_stream() if stream is None else stream
+    dev = cache.k.device
+    bufs = dev_bufs if dev_bufs is not None else {}
+
+    def up(name, t):
+        if t is None:
+            return None
+        d = bufs.get(name)
+        if d is None or d.shape != t.shape or d.dtype != t.dtype:
+            d = torch.empty(t.shape, dtype=t.dtype, device=dev)
+            bufs[name] = d
+        with torch.cuda.stream(s):
+            d.copy_(t, non_blocking=True)
+        return d
+
+    qd, wd, kd, qs = up("q", q_host), up("w", w_host), up("k_new", k_new_host), up("q_scale", q_scale_host)
+    rows = up("dst_rows", dst_rows) if not dst_rows.is_cuda else dst_rows
+    dsa_indexer_kcache_append(cache, kd, rows, stream=s)
+    T = int(np.sum(q_lens))
+    oi = bufs.get("oi")
+    if oi is None or oi.shape != (T, top_k):
+        bufs["oi"] = oi = torch.empty(T, top_k, dtype=torch.int32, device=dev)
+        bufs["os"] = torch.empty(T, top_k, dtype=torch.float32, device=dev)
+        bufs["oi_h"] = torch.empty(T, top_k, dtype=torch.int32, pin_memory=True)
+        bufs["os_h"] = torch.empty(T, top_k, dtype=torch.float32, pin_memory=True)
+    dsa_indexer_decode(qd, cache, wd, seq_lens, q_lens, top_k, q_scale=qs, k_base=k_base, out_idx=oi,
+                       out_score=bufs["os"], stream=s)
+    with torch.cuda.stream(s):
+        bufs["oi_h"].copy_(oi, non_blocking=True)
+        bufs["os_h"].copy_(bufs["os"], non_blocking=True)
+    s.synchronize()
+    return bufs["oi_h"], bufs["os_h"]

@@ -1,0 +1,90 @@
+// Internal types shared by the host planner (host_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dsa {
+
+// Device fault codes (the first one wins; reported by dsa_check_device_errors).
+enum : int {
+  DSA_DEVERR_NONE = 0,
+  DSA_DEVERR_TIMEOUT = 1,     // a bounded wait ran out
+  DSA_DEVERR_BOUNDS = 2,      // a destination row outside the cache capacity
+  DSA_DEVERR_TOPK = 3,        // selection invariant broken (count mismatch)
+};
+
+constexpr int kKeyTile = 128;       // keys per UMMA tile (the M dimension)
+constexpr int kTopkThreads = 512;   // threads per top-k CTA
+constexpr int kTopkBins = 2048;     // histogram bins per refinement level
+
+// One unit of logits work: `n_tok` consecutive query rows of one sequence against
+// key tiles [kt_begin, kt_end) of that sequence.
+struct LogitsItem {
+  int64_t k_row0;    // cache row holding key position 0 of the sequence
+  int32_t q_row0;    // global (packed) row of the item's first query
+  int32_t n_tok;     // queries in this item
+  int32_t pos0;      // position of the first query inside its sequence
+  int32_t kt_begin;  // first key tile
+  int32_t kt_end;    // one past the last key tile
+  int32_t pad;
+};
+static_assert(sizeof(LogitsItem) == 32, "LogitsItem layout");
+
+struct LogitsArgs {
+  const LogitsItem* items;
+  const int32_t* cta_items;  // [grid + 1]: items of CTA c are [cta_items[c], cta_items[c+1])
+  const int64_t* row_off;    // [T_total]: score row r starts at scores + row_off[r]
+  const float* w;            // [T_total, H]
+  const float* q_scale;      // [T_total] (FP8) or nullptr
+  const float* k_scale;      // [capacity_rows] (FP8) or nullptr
+  int64_t k_capacity;        // rows in the cache (bounds for k_scale reads)
+  float* scores;             // workspace
+  float inv_sqrt_d;
+  int* err;
+};
+
+struct TopkArgs {
+  const float* scores;
+  const int64_t* row_off;
+  const int32_t* row_pos;    // [T_total]: position p of each query row (valid keys 0..p)
+  const int32_t* rows;       // rows handled by this launch
+  int32_t n_rows;
+  int32_t top_k;
+  int32_t* out_idx;
+  float* out_score;
+  int* err;
+};
+
+// ----------------------------------------------------------------------------- launchers
+
+// Logits kernel configuration chosen by the host.
+struct LogitsLaunch {
+  int H, D;
+  bool fp8;
+  int tpa;     // queries per accumulator (N = tpa * H)
+  int ng;      // accumulators (query groups) per work item
+  int grid;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_logits(const LogitsLaunch& L, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q,
+                          const LogitsArgs& a);
+bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng);
+
+// Top-k over rows longer than top_k: one cluster of `cluster` CTAs per row,
+// `ept` keys per thread held in registers.
+cudaError_t launch_topk(const TopkArgs& a, int ept, int cluster, cudaStream_t stream);
+// Rows with at most top_k candidates: every causal position, then padding.
+cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream);
+
+cudaError_t launch_quantize_rows_fp8(const void* src, int src_is_f32, int64_t rows, int32_t row_len,
+                                     uint8_t* dst, float* scale, const int64_t* dst_rows, int64_t dst_capacity,
+                                     int* err, cudaStream_t stream);
+cudaError_t launch_append_bf16(const void* src, int src_is_f32, int64_t rows, int32_t row_len, uint16_t* dst,
+                               const int64_t* dst_rows, int64_t dst_capacity, int* err, cudaStream_t stream);
+
+int num_sms(int device);
+
+}  // namespace dsa

@@ -1,0 +1,390 @@
+// Indexer logits on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Computes, for every query row t of a work item and every key s of a 128-key
+// tile,
+//     I[t, s] = k_scale[s] * sum_h w'[t, h] * ReLU( q[t, h, :] . k[s, :] )
+//     w'[t, h] = w[t, h] * q_scale[t] / sqrt(d)
+// which is the score of page "从原理到代码：手把手教你理解DeepSeek-V3.2的闪电索引器设计"
+// §2.1 (and "Lightning Indexer 详解" §4) with one key per token shared by every head;
+// positive scales move through the ReLU unchanged.  Only keys at or before the
+// query's position are stored (the causal mask of the first page, §3 step 5); the
+// rest of a score row is never written and never read.
+//
+// Mapping ("swap AB"): the key tile is the UMMA A operand (M = 128 keys), the
+// item's queries x heads are the B operand (N = queries_per_acc * H), both
+// K-major in 128-byte-swizzled shared memory written by TMA.  The fp32
+// accumulator sits in TMEM with TMEM lane = key, so each epilogue thread owns
+// one key and reduces over heads in registers: no cross-thread reduction, and
+// score stores are coalesced along s.  The [T, H, S] logits never leave TMEM.
+//
+// Warp roles (one CTA per SM, persistent over a host-built list of work items):
+//   warp 0      TMA producer: Q block once per item, then a ring of K tiles
+//   warp 1      TMEM allocator and single-thread UMMA issuer
+//   warps 2..   epilogue: tcgen05.ld -> ReLU / weighted head sum / scale / mask -> store
+// Accumulators form a ring of TMEM buffers so the epilogue of one tile overlaps
+// the MMAs of the next.  Every wait is bounded (see ptx.cuh).
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+template <int H_, int D_, bool FP8_, int TPA_, int NG_, int NE_, int STAGES_>
+struct Cfg {
+  static constexpr int H = H_, D = D_, TPA = TPA_, NG = NG_, NE = NE_, STAGES = STAGES_;
+  static constexpr bool FP8 = FP8_;
+  static constexpr int ESZ = FP8 ? 1 : 2;
+  static constexpr int ROW_BYTES = D * ESZ;
+  static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
+  static constexpr int KB = ROW_BYTES / 128;         // 128-byte K blocks per row
+  static constexpr int KB_ELEMS = 128 / ESZ;         // elements per K block
+  static constexpr int KSTEPS = 4;                   // UMMA K steps of 32 bytes per K block
+  static constexpr int BM = kKeyTile;                // keys per tile (UMMA M)
+  static constexpr int N = TPA * H;                  // UMMA N per accumulator
+  static_assert(N % 32 == 0 && N >= 32 && N <= 256, "accumulator width");
+  static constexpr int NT = TPA * NG;                // queries per work item
+  static constexpr int ACC_COLS = N;
+  static constexpr int NBUF = (512 / N) < 4 ? (512 / N) : 4;
+  static constexpr int TMEM_COLS_RAW = NBUF * N;
+  static constexpr int TMEM_COLS = TMEM_COLS_RAW <= 32 ? 32 : TMEM_COLS_RAW <= 64 ? 64
+                                 : TMEM_COLS_RAW <= 128 ? 128 : TMEM_COLS_RAW <= 256 ? 256 : 512;
+  static constexpr int K_BLOCK_BYTES = BM * 128;     // one K block of a key tile
+  static constexpr int K_TILE_BYTES = KB * K_BLOCK_BYTES;
+  static constexpr int Q_BLOCK_BYTES = N * 128;      // one K block of one query group
+  static_assert(Q_BLOCK_BYTES % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+  static constexpr int Q_BYTES = NG * KB * Q_BLOCK_BYTES;
+  static constexpr int THREADS = (2 + NE) * 32;
+  // shared memory carve-up (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_Q = OFF_K + STAGES * K_TILE_BYTES;
+  // each epilogue warp keeps its own copy of the item's w' and score-row offsets,
+  // so the epilogue warps never wait on one another
+  static constexpr int OFF_W = OFF_Q + Q_BYTES;
+  static constexpr int W_WARP_FLOATS = NT * H;
+  static constexpr int OFF_ROW = OFF_W + NE * W_WARP_FLOATS * 4;
+  static constexpr int OFF_BAR = (OFF_ROW + NE * NT * 8 + 7) / 8 * 8;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 * NBUF + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  // + alignment slack; at least 120 KB so that one CTA holds an SM (and all its TMEM)
+  static constexpr int SMEM_RAW = OFF_MISC + 16 + 1024;
+  static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+  static constexpr uint32_t IDESC = make_idesc(FP8 ? 0u : 1u, BM, N);
+};
+
+template <class C>
+__device__ __forceinline__ void issue_umma(uint32_t d_tmem, uint32_t k_stage_addr, uint32_t q_group_addr) {
+#pragma unroll
+  for (int kb = 0; kb < C::KB; ++kb) {
+#pragma unroll
+    for (int ks = 0; ks < C::KSTEPS; ++ks) {
+      const uint64_t a = sdesc_kmajor_sw128(k_stage_addr + kb * C::K_BLOCK_BYTES + ks * 32);
+      const uint64_t b = sdesc_kmajor_sw128(q_group_addr + kb * C::Q_BLOCK_BYTES + ks * 32);
+      const uint32_t acc = (kb | ks) != 0;
+      if constexpr (C::FP8)
+        umma_f8(d_tmem, a, b, C::IDESC, acc);
+      else
+        umma_f16(d_tmem, a, b, C::IDESC, acc);
+    }
+  }
+}
+
+// sum_h w[h] * max(x[h], 0) over 32 TMEM columns starting at column `col`.
+__device__ __forceinline__ float relu_dot32(uint32_t taddr, const float* __restrict__ w) {
+  uint32_t r[32];
+  tmem_ld_32x32b_x32(taddr, r);
+  tmem_ld_wait();
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int h = 0; h < 32; h += 4) {
+    const float4 wv = *reinterpret_cast<const float4*>(w + h);
+    s0 = fmaf(wv.x, fmaxf(__uint_as_float(r[h + 0]), 0.f), s0);
+    s1 = fmaf(wv.y, fmaxf(__uint_as_float(r[h + 1]), 0.f), s1);
+    s0 = fmaf(wv.z, fmaxf(__uint_as_float(r[h + 2]), 0.f), s0);
+    s1 = fmaf(wv.w, fmaxf(__uint_as_float(r[h + 3]), 0.f), s1);
+  }
+  return s0 + s1;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+              const LogitsArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + C::STAGES;
+  uint64_t* q_full = bars + 2 * C::STAGES;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* acc_full = q_full + 2;
+  uint64_t* acc_empty = acc_full + C::NBUF;
+  uint64_t* drain = acc_empty + C::NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int item_begin = args.cta_items[blockIdx.x];
+  const int item_end = args.cta_items[blockIdx.x + 1];
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int b = 0; b < C::NBUF; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], C::NE);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t smem_base = smem_addr(smem);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_k = C::NG > 1 ? policy_evict_last() : policy_evict_first();
+      const uint64_t pol_q = policy_evict_first();
+      uint32_t k_iter = 0, item_iter = 0;
+      bool ok = true;
+      for (int it = item_begin; it < item_end && ok; ++it) {
+        const LogitsItem wi = args.items[it];
+        if (!mbar_wait(q_empty, (item_iter & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+        for (int g = 0; g < C::NG; ++g)
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(smem + C::OFF_Q + (g * C::KB + kb) * C::Q_BLOCK_BYTES, &tmap_q, q_full,
+                        kb * C::KB_ELEMS, (wi.q_row0 + g * C::TPA) * C::H, pol_q);
+        ++item_iter;
+        for (int kt = wi.kt_begin; kt < wi.kt_end; ++kt, ++k_iter) {
+          const int s = k_iter % C::STAGES;
+          if (!mbar_wait(&k_empty[s], ((k_iter / C::STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[s], C::K_TILE_BYTES);
+          const int32_t y = static_cast<int32_t>(wi.k_row0 + static_cast<int64_t>(kt) * C::BM);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(smem + C::OFF_K + s * C::K_TILE_BYTES + kb * C::K_BLOCK_BYTES, &tmap_k, &k_full[s],
+                        kb * C::KB_ELEMS, y, pol_k);
+        }
+      }
+      // Drain: the last load issued on each stage (and the last Q load) must land
+      // before this CTA may exit.  These waits end on their own; they are bounded anyway.
+      const uint32_t issued = k_iter < static_cast<uint32_t>(C::STAGES) ? k_iter : C::STAGES;
+      for (uint32_t i = 0; i < issued; ++i) {
+        const uint32_t n = k_iter - 1 - i;
+        volatile int never = 0;
+        mbar_wait(&k_full[n % C::STAGES], (n / C::STAGES) & 1, &never);
+      }
+      if (item_iter > 0) {
+        volatile int never = 0;
+        mbar_wait(q_full, (item_iter - 1) & 1, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      uint32_t k_iter = 0, acc_iter = 0, item_iter = 0;
+      bool ok = true;
+      for (int it = item_begin; it < item_end && ok; ++it) {
+        const LogitsItem wi = args.items[it];
+        const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
+        if (!mbar_wait(q_full, item_iter & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        for (int kt = wi.kt_begin; kt < wi.kt_end && ok; ++kt, ++k_iter) {
+          const int s = k_iter % C::STAGES;
+          if (!mbar_wait(&k_full[s], (k_iter / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          for (int g = 0; g < groups; ++g, ++acc_iter) {
+            const int b = acc_iter % C::NBUF;
+            if (!mbar_wait(&acc_empty[b], ((acc_iter / C::NBUF) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_umma<C>(tmem_base + b * C::ACC_COLS, smem_base + C::OFF_K + s * C::K_TILE_BYTES,
+                          smem_base + C::OFF_Q + g * C::KB * C::Q_BLOCK_BYTES);
+            umma_commit(&acc_full[b]);
+          }
+          if (ok) umma_commit(&k_empty[s]);
+        }
+        if (ok) umma_commit(q_empty);
+        ++item_iter;
+      }
+      // Let every issued UMMA finish before TMEM is released.
+      umma_commit(drain);
+      volatile int never = 0;
+      mbar_wait(drain, 0, &never);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int ew = warp - 2;                  // 0 .. NE-1
+    const int sub = warp & 3;                 // TMEM subpartition this warp may access
+    constexpr int SPLIT = C::NE / 4;          // warps sharing one subpartition
+    const int part = ew / 4;                  // which share of the queries this warp takes
+    float* wq = reinterpret_cast<float*>(smem + C::OFF_W) + ew * C::W_WARP_FLOATS;
+    int64_t* rowoff = reinterpret_cast<int64_t*>(smem + C::OFF_ROW) + ew * C::NT;
+    uint32_t acc_iter = 0;
+    bool ok = true;
+    for (int it = item_begin; it < item_end && ok; ++it) {
+      const LogitsItem wi = args.items[it];
+      __syncwarp();                           // this warp is done with the previous item's copies
+      for (int i = lane; i < wi.n_tok * C::H; i += 32) {
+        const int j = i / C::H;
+        float v = args.w[static_cast<int64_t>(wi.q_row0 + j) * C::H + (i - j * C::H)] * args.inv_sqrt_d;
+        if constexpr (C::FP8) v *= args.q_scale[wi.q_row0 + j];
+        wq[i] = v;
+      }
+      for (int j = lane; j < wi.n_tok; j += 32) rowoff[j] = args.row_off[wi.q_row0 + j];
+      __syncwarp();
+      const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
+      const int pos_last = wi.pos0 + wi.n_tok - 1;
+      for (int kt = wi.kt_begin; kt < wi.kt_end && ok; ++kt) {
+        const int key0 = kt * C::BM;                      // first key of the tile
+        const int key = key0 + sub * 32 + lane;           // this thread's key (its TMEM lane)
+        float kscale = 1.f;
+        if constexpr (C::FP8) {
+          const int64_t krow = wi.k_row0 + key;
+          kscale = (key <= pos_last && krow < args.k_capacity) ? __ldg(args.k_scale + krow) : 0.f;
+        }
+        for (int g = 0; g < groups; ++g, ++acc_iter) {
+          const int b = acc_iter % C::NBUF;
+          if (!mbar_wait(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::ACC_COLS;
+          const int j_lo = g * C::TPA;
+          const int j_hi = min(j_lo + C::TPA, wi.n_tok);
+          if constexpr (C::H >= 32) {
+            for (int j = j_lo + part; j < j_hi; j += SPLIT) {
+              if (key0 > wi.pos0 + j) continue;           // whole tile after this query: nothing to store
+              float acc = 0.f;
+#pragma unroll
+              for (int c = 0; c < C::H / 32; ++c)
+                acc += relu_dot32(tbase + (j - j_lo) * C::H + c * 32, wq + j * C::H + c * 32);
+              if (key <= wi.pos0 + j) args.scores[rowoff[j] + key] = acc * kscale;
+            }
+          } else {
+            // H < 32: one 32-column load holds 32/H queries
+            constexpr int QPC = 32 / C::H;
+            for (int c = part; c < C::N / 32; c += SPLIT) {
+              const int jc = j_lo + c * QPC;
+              if (jc >= j_hi) break;
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(tbase + c * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int u = 0; u < QPC; ++u) {
+                const int j = jc + u;
+                if (j < j_hi && key <= wi.pos0 + j) {
+                  float acc = 0.f;
+#pragma unroll
+                  for (int h = 0; h < C::H; ++h)
+                    acc = fmaf(wq[j * C::H + h], fmaxf(__uint_as_float(r[u * C::H + h]), 0.f), acc);
+                  args.scores[rowoff[j] + key] = acc * kscale;
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+      }
+    }
+  }
+
+  __syncwarp();                              // the single-lane roles rejoin their warps
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) record_error(args.err, DSA_DEVERR_TIMEOUT, blockIdx.x);
+}
+
+template <class C>
+cudaError_t launch_cfg(const LogitsLaunch& L, const CUtensorMap& tk, const CUtensorMap& tq, const LogitsArgs& a) {
+  static unsigned long long configured = 0;   // one bit per device ordinal
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(configured & (1ull << dev))) {
+    e = cudaFuncSetAttribute(logits_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured |= 1ull << dev;
+  }
+  logits_kernel<C><<<L.grid, C::THREADS, C::SMEM_BYTES, L.stream>>>(tk, tq, a);
+  return cudaGetLastError();
+}
+
+// The configurations this library is built with.  H=64/d=128 is the DeepSeek-V3.2
+// indexer shape ("Study MLA Indexer", 关键参数); H=4/d=64 serves small models.
+//                                  H   D   FP8   TPA NG NE STAGES
+using CfgPrefillBf16   = Cfg<64, 128, false, 4, 2, 8, 2>;
+using CfgPrefillFp8    = Cfg<64, 128, true,  4, 2, 8, 4>;
+using CfgDecode1Bf16   = Cfg<64, 128, false, 1, 1, 4, 6>;
+using CfgDecode2Bf16   = Cfg<64, 128, false, 2, 1, 4, 5>;
+using CfgDecode4Bf16   = Cfg<64, 128, false, 4, 1, 4, 4>;
+using CfgDecode1Fp8    = Cfg<64, 128, true,  1, 1, 4, 10>;
+using CfgDecode2Fp8    = Cfg<64, 128, true,  2, 1, 4, 10>;
+using CfgDecode4Fp8    = Cfg<64, 128, true,  4, 1, 4, 10>;
+using CfgPrefillSmallH = Cfg<4,  64,  false, 64, 1, 4, 4>;
+
+template <class... Cs>
+constexpr bool all_fit() { return ((Cs::SMEM_BYTES <= 232448) && ...); }
+static_assert(all_fit<CfgPrefillBf16, CfgPrefillFp8, CfgDecode1Bf16, CfgDecode2Bf16, CfgDecode4Bf16, CfgDecode1Fp8,
+                      CfgDecode2Fp8, CfgDecode4Fp8, CfgPrefillSmallH>(),
+              "shared memory of a configuration exceeds 227 KB");
+
+}  // namespace
+
+bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng) {
+  if (H == 64 && D == 128) {
+    if (ng == 2 && tpa == 4) return true;
+    if (ng == 1 && (tpa == 1 || tpa == 2 || tpa == 4)) return true;
+  }
+  if (H == 4 && D == 64 && !fp8 && tpa == 64 && ng == 1) return true;
+  return false;
+}
+
+cudaError_t launch_logits(const LogitsLaunch& L, const CUtensorMap& tk, const CUtensorMap& tq,
+                          const LogitsArgs& a) {
+  if (L.grid <= 0) return cudaSuccess;
+  if (L.H == 64 && L.D == 128) {
+    if (L.ng == 2 && L.tpa == 4)
+      return L.fp8 ? launch_cfg<CfgPrefillFp8>(L, tk, tq, a) : launch_cfg<CfgPrefillBf16>(L, tk, tq, a);
+    if (L.ng == 1) {
+      switch (L.tpa) {
+        case 1: return L.fp8 ? launch_cfg<CfgDecode1Fp8>(L, tk, tq, a) : launch_cfg<CfgDecode1Bf16>(L, tk, tq, a);
+        case 2: return L.fp8 ? launch_cfg<CfgDecode2Fp8>(L, tk, tq, a) : launch_cfg<CfgDecode2Bf16>(L, tk, tq, a);
+        case 4: return L.fp8 ? launch_cfg<CfgDecode4Fp8>(L, tk, tq, a) : launch_cfg<CfgDecode4Bf16>(L, tk, tq, a);
+        default: break;
+      }
+    }
+  }
+  if (L.H == 4 && L.D == 64 && !L.fp8 && L.tpa == 64 && L.ng == 1)
+    return launch_cfg<CfgPrefillSmallH>(L, tk, tq, a);
+  return cudaErrorInvalidValue;
+}
+
+int logits_queries_per_item(int H, int D, bool prefill, int max_q_len) {
+  (void)D;
+  if (H == 4) return 64;
+  if (prefill) return 8;
+  return max_q_len <= 1 ? 1 : max_q_len <= 2 ? 2 : 4;
+}
+
+}  // namespace dsa

@@ -1,0 +1,299 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Every case runs the library on seeded inputs and compares with the oracle fed the
+same bits (bf16 inputs decoded exactly; FP8 codes produced by the oracle's own
+codec, checked byte for byte against the library's append / quantise kernels).
+Small cases compare every row; the full-size workloads compare sampled rows,
+always including the first rows, the rows around the top_k boundary and the last.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_token_02_b200 import api
+from sparse_attention_token_02_b200 import workloads as W
+
+from ._parity import RTOL, Uploaded, bits_to_bf16_tensor, check_row
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    api.dsa_version()          # the CUDA library must load
+    yield
+    api.dsa_check_device_errors()
+
+
+def _run(up: Uploaded, decode: bool = False, top_k: int | None = None):
+    wl = up.wl
+    k = wl.top_k if top_k is None else top_k
+    if decode:
+        idx, sc = api.dsa_indexer_decode(up.q, up.cache, up.w, wl.seq_lens, wl.q_lens, k, q_scale=up.q_scale,
+                                         k_base=up.k_base)
+    else:
+        idx, sc = api.dsa_indexer_prefill(up.q, up.cache, up.w, wl.seq_lens, k, q_scale=up.q_scale,
+                                          q_lens=wl.q_lens, k_base=up.k_base)
+    api.dsa_check_device_errors()
+    return idx.cpu().numpy(), sc.cpu().numpy()
+
+
+def _sample_rows(wl: W.Workload, n_mid: int = 8, seed: int = 0):
+    T = wl.total_q
+    rng = np.random.default_rng(seed)
+    picks = {0, 1, T - 1, T - 2}
+    k = wl.top_k
+    seq_pos = []
+    for Lb, n in zip(wl.seq_lens, wl.q_lens):
+        seq_pos += list(range(Lb - n, Lb))
+    seq_pos = np.array(seq_pos)
+    for target in (k - 2, k - 1, k, k + 1, 2 * k + 5):
+        hit = np.nonzero(seq_pos == target)[0]
+        if hit.size:
+            picks.add(int(hit[0]))
+    picks.update(int(x) for x in rng.integers(0, T, size=n_mid))
+    return sorted(p for p in picks if 0 <= p < T)
+
+
+def _check(up: Uploaded, idx, sc, rows, top_k=None):
+    k = up.wl.top_k if top_k is None else top_k
+    rtol = RTOL[up.wl.dtype]
+    orows = up.oracle_rows(rows)
+    for r, orow in zip(rows, orows):
+        check_row(idx[r], sc[r], orow, k, rtol, what=f"{up.wl.name} row {r}")
+
+
+# ----------------------------------------------------------------------------- append / quantise (a1)
+
+def test_append_bf16_copy_and_f32_rounding():
+    rng = np.random.default_rng(0)
+    src32 = (rng.standard_normal((300, 128)) * 3).astype(np.float32)
+    cache = api.IndexerKCache.empty(1000, 128, fp8=False)
+    rows = torch.from_numpy(rng.permutation(1000)[:300].astype(np.int64)).cuda()
+    api.dsa_indexer_kcache_append(cache, torch.from_numpy(src32).cuda(), rows)
+    got = cache.k[rows].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, W.f32_to_bf16_bits(src32))
+    bits = W.f32_to_bf16_bits(src32[::-1].copy())
+    api.dsa_indexer_kcache_append(cache, bits_to_bf16_tensor(bits), rows)
+    got = cache.k[rows].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, bits)
+    api.dsa_check_device_errors()
+
+
+@pytest.mark.parametrize("row_len", [128, 8192])
+def test_quantize_rows_fp8_bit_exact_against_oracle_codec(row_len):
+    rng = np.random.default_rng(row_len)
+    x = (rng.standard_normal((257, row_len)) * rng.uniform(1e-3, 50, (257, 1))).astype(np.float32)
+    x[3] = 0.0
+    x[4, :7] = [1e-8, -1e-8, 3e4, -3e4, 0.0, 1.0, -1.0]
+    bits = W.f32_to_bf16_bits(x)
+    codes, scale = api.dsa_quantize_rows_fp8(bits_to_bf16_tensor(bits))
+    ref_codes, ref_scale = oracle.quantize_rows(oracle.bf16_bits_to_f64(bits).astype(np.float32))
+    assert np.array_equal(scale.cpu().numpy(), ref_scale)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    # fp32 sources too
+    codes, scale = api.dsa_quantize_rows_fp8(torch.from_numpy(x).cuda())
+    ref_codes, ref_scale = oracle.quantize_rows(x)
+    assert np.array_equal(scale.cpu().numpy(), ref_scale)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+
+
+def test_fp8_cache_append_matches_oracle_codec():
+    wl = W.scaled(W.decode8(), seq_lens=(700, 333), q_lens=(2, 2))
+    up = Uploaded(wl)
+    for b in range(2):
+        lo = int(up.k_base[b])
+        codes, scale = oracle.quantize_rows(oracle.bf16_bits_to_f64(up.inp["k_bits"][b]).astype(np.float32))
+        got = up.cache.k[lo: lo + wl.seq_lens[b]].cpu().numpy()
+        gs = up.cache.k_scale[lo: lo + wl.seq_lens[b]].cpu().numpy()
+        assert np.array_equal(got, codes) and np.array_equal(gs, scale)
+
+
+def test_append_out_of_range_row_is_reported_and_skipped():
+    cache = api.IndexerKCache.empty(16, 128, fp8=True)
+    src = torch.ones(2, 128, dtype=torch.bfloat16, device="cuda")
+    api.dsa_indexer_kcache_append(cache, src, torch.tensor([3, 16], dtype=torch.int64, device="cuda"))
+    with pytest.raises(RuntimeError, match="DEVICE_CHECK"):
+        api.dsa_check_device_errors()
+    assert int(cache.k[3, 0]) != 0          # the valid row was written
+    api.dsa_check_device_errors()           # the flag was cleared
+
+
+# ----------------------------------------------------------------------------- prefill
+
+def test_tiny_workload_all_rows_and_dense_scores():
+    wl = W.tiny()
+    up = Uploaded(wl)
+    idx, sc = _run(up)
+    rows = list(range(wl.total_q))
+    _check(up, idx, sc, rows)
+    dense = api.dsa_indexer_scores(up.q, up.cache, up.w, wl.seq_lens, k_base=up.k_base).cpu().numpy()
+    for r, orow in zip(rows, up.oracle_rows(rows)):
+        p = orow.shape[0]
+        o_k = np.sort(orow)[::-1][min(wl.top_k, p) - 1]
+        tol = RTOL["bf16"] * np.maximum(np.abs(orow), max(abs(o_k), 1e-30))
+        assert np.all(np.abs(dense[r, :p] - orow) <= tol), f"row {r}"
+        assert np.all(np.isneginf(dense[r, p:]))
+
+
+def test_prefill_bf16_ragged_batch_chunked_and_offset_cache():
+    # three sequences: a full prefill, a chunked prefill (q_len < seq_len) and a single query;
+    # the cache rows of the sequences are not packed (k_base with gaps)
+    wl = W.scaled(W.prefill(), seq_lens=(700, 450, 129), q_lens=(700, 200, 1), top_k=256, outlier_frac=0.01)
+    inp = W.make_inputs(wl)
+    up = Uploaded(wl, inp)
+    base = np.array([5000, 37, 2000], dtype=np.int64)
+    cache = api.IndexerKCache.empty(6000, 128, fp8=False)
+    for b in range(3):
+        rows = torch.arange(base[b], base[b] + wl.seq_lens[b], dtype=torch.int64, device="cuda")
+        api.dsa_indexer_kcache_append(cache, bits_to_bf16_tensor(inp["k_bits"][b]), rows)
+    idx, sc = api.dsa_indexer_prefill(up.q, cache, up.w, wl.seq_lens, wl.top_k, q_lens=wl.q_lens, k_base=base)
+    api.dsa_check_device_errors()
+    _check(up, idx.cpu().numpy(), sc.cpu().numpy(), list(range(wl.total_q)))
+
+
+def test_prefill_bf16_top_k_2048_boundary_rows():
+    wl = W.scaled(W.prefill(), seq_lens=(2600,), q_lens=(2600,))
+    up = Uploaded(wl)
+    idx, sc = _run(up)
+    rows = _sample_rows(wl, n_mid=10) + list(range(2040, 2060))
+    _check(up, idx, sc, sorted(set(rows)))
+
+
+def test_prefill_fp8_small():
+    wl = W.scaled(W.prefill8(), seq_lens=(2300, 517), q_lens=(2300, 517))
+    up = Uploaded(wl)
+    idx, sc = _run(up)
+    _check(up, idx, sc, _sample_rows(wl, n_mid=12) + list(range(2300, 2310)))
+
+
+# ----------------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("q_len", [1, 2, 3])
+def test_decode_bf16_ragged(q_len):
+    lens = (5000, 130, 2049, q_len, 4096, 33, 2051)
+    wl = W.scaled(W.decode(), seq_lens=lens, q_lens=(q_len,) * len(lens), seed=10 + q_len)
+    up = Uploaded(wl)
+    idx, sc = _run(up, decode=True)
+    _check(up, idx, sc, list(range(wl.total_q)))
+
+
+def test_decode_fp8_ragged_pairs():
+    wl = W.scaled(W.decode8(), seq_lens=(9000, 2049, 4097, 3000, 2), q_lens=(2,) * 5)
+    up = Uploaded(wl)
+    idx, sc = _run(up, decode=True)
+    _check(up, idx, sc, list(range(wl.total_q)))
+
+
+def test_decode_row_equals_prefill_row():
+    wl = W.scaled(W.prefill(), seq_lens=(3000,), q_lens=(3000,), outlier_frac=0.0)
+    up = Uploaded(wl)
+    pidx, psc = _run(up)
+    last = slice(2998, 3000)
+    q_dec = up.q[last].contiguous()
+    w_dec = up.w[last].contiguous()
+    didx, dsc = api.dsa_indexer_decode(q_dec, up.cache, w_dec, (3000,), (2,), wl.top_k, k_base=up.k_base)
+    didx, dsc = didx.cpu().numpy(), dsc.cpu().numpy()
+    for j, r in enumerate((2998, 2999)):
+        a = np.sort(pidx[r][pidx[r] >= 0])
+        b = np.sort(didx[j][didx[j] >= 0])
+        assert np.array_equal(a, b)
+        order_a, order_b = np.argsort(pidx[r]), np.argsort(didx[j])
+        np.testing.assert_allclose(psc[r][order_a], dsc[j][order_b], rtol=1e-6, atol=0)
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+def test_edge_top_k_larger_than_every_row_and_top_k_one():
+    wl = W.scaled(W.prefill(), seq_lens=(300, 1), q_lens=(300, 1), top_k=512)
+    up = Uploaded(wl)
+    idx, sc = _run(up)
+    _check(up, idx, sc, list(range(wl.total_q)))
+    idx1, sc1 = _run(up, top_k=1)
+    _check(up, idx1, sc1, list(range(wl.total_q)), top_k=1)
+
+
+def test_edge_ties_and_zero_and_negative_weights():
+    wl = W.scaled(W.prefill(), seq_lens=(1500,), q_lens=(1500,), top_k=100)
+    inp = W.make_inputs(wl)
+    # integer-valued keys and queries: many exactly equal scores
+    rng = np.random.default_rng(1)
+    inp["k_bits"] = [W.f32_to_bf16_bits(rng.integers(-2, 3, (1500, 128)).astype(np.float32))]
+    inp["q_bits"] = W.f32_to_bf16_bits(rng.integers(-1, 2, (1500, 64, 128)).astype(np.float32))
+    for w in (np.full((1500, 64), 1.0 / 64, np.float32),
+              np.zeros((1500, 64), np.float32),
+              rng.standard_normal((1500, 64)).astype(np.float32)):
+        inp["w"] = w
+        up = Uploaded(wl, inp)
+        idx, sc = _run(up)
+        _check(up, idx, sc, [0, 1, 99, 100, 101, 500, 1499])
+
+
+def test_edge_empty_batch_and_zero_query_sequences():
+    wl = W.scaled(W.prefill(), seq_lens=(40, 10), q_lens=(0, 10), top_k=16)
+    up = Uploaded(wl)
+    idx, sc = _run(up)
+    _check(up, idx, sc, list(range(10)))
+    q = torch.zeros(0, 64, 128, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(0, 64, dtype=torch.float32, device="cuda")
+    i0, s0 = api.dsa_indexer_prefill(q, up.cache, w, [], 16)
+    assert i0.shape == (0, 16)
+
+
+def test_edge_invalid_arguments_raise():
+    up = Uploaded(W.scaled(W.decode(), seq_lens=(300,), q_lens=(1,)))
+    with pytest.raises(RuntimeError, match="INVALID_ARG"):
+        api.dsa_indexer_decode(up.q, up.cache, up.w, (300,), (5,), 16)       # q_len > 4
+    with pytest.raises(RuntimeError, match="INVALID_ARG"):
+        api.dsa_indexer_prefill(up.q, up.cache, up.w, (300,), 0, q_lens=(1,))  # top_k = 0
+    with pytest.raises(RuntimeError, match="INVALID_ARG"):
+        api.dsa_indexer_prefill(up.q, up.cache, up.w, (10 ** 6,), 16, q_lens=(1,))  # beyond capacity
+    q32 = torch.zeros(1, 32, 128, dtype=torch.bfloat16, device="cuda")
+    w32 = torch.zeros(1, 32, dtype=torch.float32, device="cuda")
+    with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+        api.dsa_indexer_prefill(q32, up.cache, w32, (300,), 16, q_lens=(1,))
+
+
+# ----------------------------------------------------------------------------- full-size workloads (sampled rows)
+
+def test_full_decode_batch_all_rows():
+    wl = W.decode()
+    up = Uploaded(wl)
+    idx, sc = _run(up, decode=True)
+    _check(up, idx, sc, list(range(wl.total_q)))
+
+
+def test_full_prefill_bf16_sampled_rows():
+    wl = W.prefill()
+    up = Uploaded(wl)
+    idx, sc = _run(up)
+    _check(up, idx, sc, _sample_rows(wl, n_mid=10))
+
+
+def test_full_prefill_fp8_sampled_rows():
+    wl = W.prefill8()
+    up = Uploaded(wl)
+    # the library's FP8 codes for the sampled query rows equal the oracle codec's
+    rows = _sample_rows(wl, n_mid=8)
+    bits = up.inp["q_bits"][rows].reshape(len(rows), -1)
+    codes, scale = oracle.quantize_rows(oracle.bf16_bits_to_f64(bits).astype(np.float32))
+    assert np.array_equal(up.q[rows].reshape(len(rows), -1).cpu().numpy(), codes)
+    assert np.array_equal(up.q_scale[rows].cpu().numpy(), scale)
+    idx, sc = _run(up)
+    _check(up, idx, sc, rows)
+
+
+def test_full_ragged_decode_fp8_sampled_sequences():
+    wl = W.decode8()
+    up = Uploaded(wl)
+    idx, sc = _run(up, decode=True)
+    order = np.argsort(wl.seq_lens)
+    seqs = [int(order[0]), int(order[-1]), int(order[len(order) // 2])]
+    rows = sorted(2 * b + j for b in seqs for j in (0, 1))
+    _check(up, idx, sc, rows)
