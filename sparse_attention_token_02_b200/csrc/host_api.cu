@@ -594,12 +594,14 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   la.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   la.err = c->d_err;
   LogitsLaunch L{H, D, fp8, tpa, ng, static_cast<int>(p.cta_items.size()) - 1, stream};
-  if (g_prof[0]) DSA_CUDA_TRY(cudaEventRecord(g_prof[0], stream), "cudaEventRecord");
+  // inside a capture the events must become event-record nodes of the graph
+  const unsigned ev_flags = capturing ? cudaEventRecordExternal : cudaEventRecordDefault;
+  if (g_prof[0]) DSA_CUDA_TRY(cudaEventRecordWithFlags(g_prof[0], stream, ev_flags), "cudaEventRecord");
   DSA_CUDA_TRY(launch_logits(L, tk, tq, la), "logits kernel launch");
   g_launches += L.grid > 0;
-  if (g_prof[1]) DSA_CUDA_TRY(cudaEventRecord(g_prof[1], stream), "cudaEventRecord");
+  if (g_prof[1]) DSA_CUDA_TRY(cudaEventRecordWithFlags(g_prof[1], stream, ev_flags), "cudaEventRecord");
   if (mode == Mode::Scores) {
-    if (g_prof[2]) DSA_CUDA_TRY(cudaEventRecord(g_prof[2], stream), "cudaEventRecord");
+    if (g_prof[2]) DSA_CUDA_TRY(cudaEventRecordWithFlags(g_prof[2], stream, ev_flags), "cudaEventRecord");
     return DSA_OK;
   }
 
@@ -626,7 +628,7 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     DSA_CUDA_TRY(launch_topk(s, cl.ept, cl.cluster, stream), "top-k launch");
     ++g_launches;
   }
-  if (g_prof[2]) DSA_CUDA_TRY(cudaEventRecord(g_prof[2], stream), "cudaEventRecord");
+  if (g_prof[2]) DSA_CUDA_TRY(cudaEventRecordWithFlags(g_prof[2], stream, ev_flags), "cudaEventRecord");
   return DSA_OK;
 }
 
