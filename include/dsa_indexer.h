@@ -164,6 +164,33 @@ DSA_API dsa_status_t dsa_indexer_decode(const dsa_query_t* q, const dsa_kcache_t
 DSA_API dsa_status_t dsa_indexer_scores(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
                                 const dsa_batch_t* batch, float* out_scores, int64_t ld, void* stream);
 
+/*
+ * Decode that allocates no device memory.  (The pages have no counterpart: this
+ * is a library entry point for callers that may not allocate.)
+ *
+ * Same arguments and result as dsa_indexer_decode, for callers that must not
+ * allocate device memory at all: a server whose device memory belongs to its own
+ * pool, code under a device-memory budget enforced outside CUDA, or a host that
+ * forbids allocator calls on its hot path.  dsa_indexer_decode grows a workspace
+ * with cudaMalloc; this call instead keeps the score rows and the scheduling tables
+ * in one static 16 MiB __device__ array inside the library, which every GPU that
+ * loads the library holds until the process exits.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *   fault  optional device int32[2]: zeroed by the call, then receives the first
+ *          device fault (code, info) as dsa_check_device_errors would report it;
+ *          with NULL, faults are kept in the static array and not reported.
+ * Limits: the batch must fit the array: 4 bytes per cached key of every query
+ * (rounded up to 4 keys per query) plus its tables, else DSA_ERR_INVALID_ARG says
+ * how much it needs.  Every call shares the one array (per device) and leaves its
+ * contents behind, so calls that overlap on the GPU (other streams, other host
+ * threads) race; serialise them.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.
+ */
+DSA_API dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                                const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx,
+                                                float* out_score, int32_t* fault, void* stream);
+
 /* Workspace bytes a call with this batch needs (scores plus scheduling tables). */
 DSA_API size_t dsa_indexer_workspace_bytes(const dsa_query_t* q, const dsa_batch_t* batch, int32_t top_k);
 

@@ -22,6 +22,7 @@ EXPORTED = (
     "dsa_quantize_rows_fp8",
     "dsa_indexer_prefill",
     "dsa_indexer_decode",
+    "dsa_indexer_decode_noalloc",
     "dsa_indexer_scores",
     "dsa_indexer_workspace_bytes",
     "dsa_set_workspace",
@@ -76,6 +77,8 @@ def load() -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.argtypes = [P(Query), P(KCache), V, P(Batch), I32, V, V, V]
         fn.restype = st
+    lib.dsa_indexer_decode_noalloc.argtypes = [P(Query), P(KCache), V, P(Batch), I32, V, V, V, V]
+    lib.dsa_indexer_decode_noalloc.restype = st
     lib.dsa_indexer_scores.argtypes = [P(Query), P(KCache), V, P(Batch), V, I64, V]
     lib.dsa_indexer_scores.restype = st
     lib.dsa_indexer_workspace_bytes.argtypes = [P(Query), P(Batch), I32]

@@ -144,6 +144,29 @@ def dsa_indexer_decode(q, cache: IndexerKCache, w, seq_lens, q_lens, top_k, q_sc
                 stream)
 
 
+def dsa_indexer_decode_noalloc(q, cache: IndexerKCache, w, seq_lens, q_lens, top_k, q_scale=None, k_base=None,
+                               out_idx=None, out_score=None, fault=None, stream=None):
+    """dsa_indexer_decode for callers that may not allocate device memory: the library
+    keeps its scratch in a fixed static device array (16 MiB per device) instead of a
+    cudaMalloc'd workspace.  ``fault`` (optional int32 [2] CUDA tensor) receives the
+    first device fault.  Calls that overlap on the GPU share that array and race."""
+    b = _HostBatch(seq_lens, q_lens, k_base)
+    T = b.total_q
+    _require_cuda(w, fault)
+    if w.dtype != torch.float32:
+        raise TypeError("w must be fp32")
+    if out_idx is None:
+        out_idx = torch.empty(T, top_k, dtype=torch.int32, device=q.device)
+    if out_score is None:
+        out_score = torch.empty(T, top_k, dtype=torch.float32, device=q.device)
+    _require_cuda(out_idx, out_score)
+    qq, kc = _query(q, q_scale), cache.c()
+    check(_lib.load().dsa_indexer_decode_noalloc(ctypes.byref(qq), ctypes.byref(kc), _ptr(w), ctypes.byref(b.c),
+                                                 top_k, _ptr(out_idx), _ptr(out_score), _ptr(fault),
+                                                 _stream(stream)))
+    return out_idx, out_score
+
+
 def dsa_indexer_scores(q, cache: IndexerKCache, w, seq_lens, q_scale=None, q_lens=None, k_base=None, ld=None,
                        out=None, stream=None):
     """Dense scores [T_total, ld] (entries after each query's position are left as they were: -inf here)."""

@@ -772,3 +772,134 @@ const char* dsa_get_last_error(void) { return g_last_error.c_str(); }
 const char* dsa_version(void) { return "dsa_indexer 0.1 (sm_100a)"; }
 
 }  // extern "C"
+
+// ============================================================================= decode without device allocation
+//
+// dsa_indexer_decode obtains its workspace with cudaMalloc the first time a stream
+// needs it.  Some callers may not allocate at all: a serving process whose device
+// memory is carved up in advance by its own pool (an allocation behind its back can
+// fail or fragment that pool), code that runs under a device-memory budget enforced
+// outside CUDA, or an embedding that forbids allocator calls on its hot path.  For
+// them, dsa_indexer_decode_noalloc keeps the score rows and scheduling tables in one
+// file-scope __device__ array instead.  The array is part of this library's device
+// image, so every GPU that loads the library holds it until the process exits.
+
+namespace dsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB on every device
+constexpr size_t kNoAllocFaultBytes = 256;                  // fault words at the front of the array
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array on the current device.  In host code the symbol is
+// only a stand-in, so the address is looked up once per device with that device
+// current, and kept.
+dsa_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  DSA_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+  static std::mutex mu;
+  static std::map<int, void*> addr;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = addr.find(dev);
+  if (it == addr.end()) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    if (p == nullptr) return fail(DSA_ERR_CUDA, "cudaGetSymbolAddress(static scratch) returned NULL");
+    it = addr.emplace(dev, p).first;
+  }
+  *out = it->second;
+  return DSA_OK;
+}
+
+}  // namespace
+}  // namespace dsa
+
+extern "C" dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                                   const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx,
+                                                   float* out_score, int32_t* fault, void* stream_v) {
+  using namespace dsa;
+  g_last_error.clear();
+  dsa_status_t st = check_cache(kc);
+  if (st != DSA_OK) return st;
+  BatchView v;
+  if ((st = check_batch(batch, kc, true, &v)) != DSA_OK) return st;
+  if (top_k < 1) return fail(DSA_ERR_INVALID_ARG, "top_k must be >= 1");
+  if (v.total_q == 0) return DSA_OK;
+  if ((st = check_query(q, kc)) != DSA_OK) return st;
+  if (!w) return fail(DSA_ERR_INVALID_ARG, "w is NULL");
+  if (!out_idx || !out_score) return fail(DSA_ERR_INVALID_ARG, "out_idx / out_score is NULL");
+  const bool fp8 = kc->dtype == DSA_FP8_E4M3;
+  const int H = q->H_I, D = kc->d_I;
+  const int tpa = logits_queries_per_item(H, D, false, v.max_q_len);
+  if (!logits_config_supported(H, D, fp8, tpa, 1))
+    return fail(DSA_ERR_UNSUPPORTED, "no decode kernel for H_I=%d, d_I=%d, dtype=%s", H, D, fp8 ? "fp8" : "bf16");
+
+  int dev = 0;
+  DSA_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+  const int sms = num_sms(dev);
+  Plan p;
+  p.tpa = tpa;
+  p.ng = 1;
+  plan_rows(v, false, 0, &p);
+  plan_decode_items(v, sms, &p);
+  if ((st = plan_topk(v, top_k, sms, &p)) != DSA_OK) return st;
+  const MetaLayout m = layout_of(p);
+  const size_t need = kNoAllocFaultBytes + align_up(m.total) + align_up(size_t(p.score_elems) * sizeof(float));
+  if (need > kNoAllocScratchBytes)
+    return fail(DSA_ERR_INVALID_ARG,
+                "this batch needs %zu bytes of scratch; dsa_indexer_decode_noalloc has a fixed %zu "
+                "(score rows take 4 bytes per cached key, rounded up to 4 keys per query)",
+                need, kNoAllocScratchBytes);
+
+  void* base = nullptr;
+  if ((st = noalloc_scratch(&base)) != DSA_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  int* err = fault ? reinterpret_cast<int*>(fault) : static_cast<int*>(base);
+  DSA_CUDA_TRY(cudaMemsetAsync(err, 0, 2 * sizeof(int), stream), "cudaMemsetAsync(fault words)");
+  char* mb = static_cast<char*>(base) + kNoAllocFaultBytes;
+  float* d_scores = reinterpret_cast<float*>(mb + align_up(m.total));
+  // the tables come from pageable host memory: the driver stages the copy, nothing is allocated here
+  const std::vector<uint8_t> blob = pack(p, m);
+  DSA_CUDA_TRY(cudaMemcpyAsync(mb, blob.data(), blob.size(), cudaMemcpyHostToDevice, stream), "cudaMemcpyAsync");
+
+  CUtensorMap tk, tq;
+  if ((st = encode_rows(&tk, kc->k, fp8, kc->capacity_rows, D, kKeyTile)) != DSA_OK) return st;
+  if ((st = encode_rows(&tq, q->data, fp8, v.total_q * H, D, tpa * H)) != DSA_OK) return st;
+  LogitsArgs la{};
+  la.items = reinterpret_cast<const LogitsItem*>(mb + m.items);
+  la.cta_items = reinterpret_cast<const int32_t*>(mb + m.cta);
+  la.row_off = reinterpret_cast<const int64_t*>(mb + m.row_off);
+  la.w = w;
+  la.q_scale = fp8 ? q->scale : nullptr;
+  la.k_scale = fp8 ? kc->k_scale : nullptr;
+  la.k_capacity = kc->capacity_rows;
+  la.scores = d_scores;
+  la.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  la.err = err;
+  LogitsLaunch L{H, D, fp8, tpa, 1, static_cast<int>(p.cta_items.size()) - 1, stream};
+  DSA_CUDA_TRY(launch_logits(L, tk, tq, la), "logits kernel launch");
+  TopkArgs ta{};
+  ta.scores = d_scores;
+  ta.row_off = la.row_off;
+  ta.row_pos = reinterpret_cast<const int32_t*>(mb + m.row_pos);
+  ta.top_k = top_k;
+  ta.out_idx = out_idx;
+  ta.out_score = out_score;
+  ta.err = err;
+  const int32_t* rows = reinterpret_cast<const int32_t*>(mb + m.topk_rows);
+  if (p.short_count) {
+    TopkArgs s = ta;
+    s.rows = rows + p.short_first;
+    s.n_rows = static_cast<int32_t>(p.short_count);
+    DSA_CUDA_TRY(launch_topk_short(s, stream), "top-k (short rows) launch");
+  }
+  for (const auto& cl : p.classes) {
+    TopkArgs s = ta;
+    s.rows = rows + cl.first;
+    s.n_rows = static_cast<int32_t>(cl.count);
+    DSA_CUDA_TRY(launch_topk(s, cl.ept, cl.cluster, stream), "top-k launch");
+  }
+  return DSA_OK;
+}
