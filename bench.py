@@ -34,7 +34,14 @@ sys.path.insert(0, ROOT)
 
 METRIC = "indexer query-key pairs scored+selected/sec (prefill & decode); % of roofline"
 UNIT = "pairs/s"
-WORKLOAD = "decode batch: 32 seqs x 32768 keys, H_I=64, d_I=128, bf16, top_k=2048, 1 query/seq"
+WORKLOADS = {
+    "decode": "decode batch: 32 seqs x 32768 keys, H_I=64, d_I=128, bf16, top_k=2048, 1 query/seq",
+    "prefill": "prefill: 1 seq L=16384, H_I=64, d_I=128, bf16, 1% outlier keys x4, causal, top_k=2048",
+    "prefill8": "long prefill FP8: 1 seq L=65536, H_I=64, d_I=128, E4M3 + per-token scale, causal, top_k=2048",
+    "decode8": "ragged decode FP8: 16 seqs, lengths U[4096,131072], 2 queries/seq, H_I=64, d_I=128, top_k=2048",
+    "tiny": "tiny prefill: 1 seq L=512, H_I=4, d_I=64, bf16, top_k=32",
+}
+WORKLOAD = WORKLOADS["decode"]
 
 
 def parse():
@@ -47,14 +54,22 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work for the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["decode", "prefill", "prefill8", "decode8", "tiny"], default="decode",
+                    help="decode (the default) is the measured workload; the others are for profiling")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="profiling only: run a prefill workload at this sequence length instead")
     return ap.parse_args()
 
 
 # ----------------------------------------------------------------------------- workload
 
-def workload(rank: int):
+def workload(rank: int, name: str = "decode"):
+    """The workload each rank processes; ranks draw different seeds (weak scaling)."""
     from sparse_attention_token_02_b200 import workloads as W
-    return W.decode(seed=2 + 1000 * rank)
+    make = {"decode": W.decode, "prefill": W.prefill, "prefill8": W.prefill8, "decode8": W.decode8,
+            "tiny": W.tiny}[name]
+    wl = make()
+    return W.scaled(wl, seed=wl.seed + 1000 * rank) if rank else wl
 
 
 def host_inputs(wl):
@@ -202,12 +217,16 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- our path
 
 def peaks():
+    """Roofline denominators: the measured copy bandwidth and cuBLAS bf16 GEMM
+    rates (FP8 taken as 2x bf16, the nominal dense ratio), else the recipe's fallback."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        hbm, b, bs, kind = float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
     except Exception:
-        return 6650.0, "fallback"
+        hbm, b, bs, kind = 6650.0, 1590.0, 1400.0, "fallback"
+    return {"hbm": hbm, "bf16_burst": b, "bf16_sustained": bs, "fp8_burst": 2 * b, "fp8_sustained": 2 * bs,
+            "kind": kind}
 
 
 def profiled_traffic():
@@ -225,6 +244,85 @@ def profiled_traffic():
         return float(fields["dram_bytes_per_launch"].strip())
     except Exception:
         return None
+
+
+class Harness:
+    """Device state and one step of the hot path for a workload.
+
+    decode : the step appends each sequence's newest q_len keys (re-written in place),
+             quantises the queries (FP8), then scores + selects (dsa_indexer_decode).
+    prefill: the step appends every key of the sequence (quantising for FP8),
+             quantises the queries (FP8), then scores + selects (dsa_indexer_prefill).
+    """
+
+    def __init__(self, wl, inp, dev, stream):
+        import torch
+        from sparse_attention_token_02_b200 import api
+        self.api, self.wl, self.dev, self.stream = api, wl, dev, stream
+        self.fp8 = wl.dtype == "fp8"
+        self.decode = wl.kind == "decode"
+        L = np.array(wl.seq_lens, dtype=np.int64)
+        self.k_base = np.concatenate([[0], np.cumsum(L)[:-1]]).astype(np.int64)
+        self.seq_lens, self.q_lens = list(wl.seq_lens), list(wl.q_lens)
+        T, H, d = wl.total_q, wl.H, wl.d
+        bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+        with torch.cuda.stream(stream):
+            self.cache = api.IndexerKCache.empty(wl.total_k, d, self.fp8, device=dev)
+            k_all = bf(np.concatenate(inp["k_bits"])).to(dev)
+            api.dsa_indexer_kcache_append(self.cache, k_all, torch.arange(wl.total_k, dtype=torch.int64, device=dev),
+                                          stream=stream)
+            if self.decode:
+                # the step's new keys: the newest q_len rows of each sequence
+                rows = np.concatenate([self.k_base[b] + np.arange(L[b] - n, L[b]) for b, n in enumerate(self.q_lens)])
+                self.k_step_host = bf(np.concatenate(inp["k_bits"])[rows])
+                self.rows_host = torch.from_numpy(rows.astype(np.int64))
+                del k_all
+            else:
+                self.k_step_host = bf(np.concatenate(inp["k_bits"]))
+                self.rows_host = torch.arange(wl.total_k, dtype=torch.int64)
+            self.k_step = self.k_step_host.to(dev)
+            self.rows = self.rows_host.to(dev)
+            self.q_src_host = bf(inp["q_bits"])
+            self.q_src = self.q_src_host.to(dev)
+            self.w_host = torch.from_numpy(inp["w"])
+            self.w = self.w_host.to(dev)
+            if self.fp8:
+                self.q = torch.empty(T, H, d, dtype=torch.uint8, device=dev)
+                self.q_scale = torch.empty(T, dtype=torch.float32, device=dev)
+            else:
+                self.q, self.q_scale = self.q_src, None
+            self.out_idx = torch.empty(T, wl.top_k, dtype=torch.int32, device=dev)
+            self.out_score = torch.empty(T, wl.top_k, dtype=torch.float32, device=dev)
+        stream.synchronize()
+
+    def step(self, k_step=None, q_src=None, w=None):
+        api, s, wl = self.api, self.stream, self.wl
+        k_step = self.k_step if k_step is None else k_step
+        q_src = self.q_src if q_src is None else q_src
+        w = self.w if w is None else w
+        api.dsa_indexer_kcache_append(self.cache, k_step, self.rows, stream=s)
+        if self.fp8:
+            api.dsa_quantize_rows_fp8(q_src.view(q_src.shape[0], -1), dst=self.q.view(self.q.shape[0], -1),
+                                      scale=self.q_scale, stream=s)
+        q = self.q if self.fp8 else q_src
+        if self.decode:
+            api.dsa_indexer_decode(q, self.cache, w, self.seq_lens, self.q_lens, wl.top_k, q_scale=self.q_scale,
+                                   k_base=self.k_base, out_idx=self.out_idx, out_score=self.out_score, stream=s)
+        else:
+            api.dsa_indexer_prefill(q, self.cache, w, self.seq_lens, wl.top_k, q_scale=self.q_scale,
+                                    q_lens=self.q_lens, k_base=self.k_base, out_idx=self.out_idx,
+                                    out_score=self.out_score, stream=s)
+
+    # algorithmic work of the dominant (logits) kernel per step
+    def logits_bytes(self):
+        wl = self.wl
+        esz = 1 if self.fp8 else 2
+        k_bytes = wl.total_k * wl.d * esz + (wl.total_k * 4 if self.fp8 else 0)
+        q_bytes = wl.total_q * wl.H * wl.d * esz + (wl.total_q * 4 if self.fp8 else 0)
+        return k_bytes + q_bytes + wl.total_q * wl.H * 4
+
+    def logits_flops(self):
+        return 2.0 * self.wl.pairs * self.wl.H * self.wl.d
 
 
 def run_ours(args):
@@ -246,36 +344,17 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.Stream(device=dev)
 
-    wl = workload(rank)
+    wl = workload(rank, args.workload)
+    if args.seq_len and wl.kind == "prefill":
+        from sparse_attention_token_02_b200 import workloads as W
+        wl = W.scaled(wl, seq_lens=(args.seq_len,), q_lens=(args.seq_len,))
     inp = host_inputs(wl)
-    S, L, H, d, k = wl.num_seqs, wl.seq_lens[0], wl.H, wl.d, wl.top_k
-    k_base = np.arange(S, dtype=np.int64) * L
-    seq_lens, q_lens = [L] * S, [1] * S
-
-    with torch.cuda.stream(stream):
-        cache = api.IndexerKCache.empty(S * L, d, fp8=False, device=dev)
-        k_all = torch.from_numpy(np.concatenate(inp["k_bits"]).view(np.int16)).view(torch.bfloat16).to(dev)
-        api.dsa_indexer_kcache_append(cache, k_all, torch.arange(S * L, dtype=torch.int64, device=dev), stream=stream)
-        del k_all
-        q = torch.from_numpy(inp["q_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
-        w = torch.from_numpy(inp["w"]).to(dev)
-        # the step's new key of each sequence: its last cache row (re-appended every step)
-        k_new_bits = np.stack([kb[-1] for kb in inp["k_bits"]])
-        k_new = torch.from_numpy(k_new_bits.view(np.int16)).view(torch.bfloat16).to(dev)
-        dst_rows = torch.from_numpy(k_base + L - 1).to(dev)
-        out_idx = torch.empty(S, k, dtype=torch.int32, device=dev)
-        out_score = torch.empty(S, k, dtype=torch.float32, device=dev)
-    stream.synchronize()
-
-    def step():
-        api.dsa_indexer_kcache_append(cache, k_new, dst_rows, stream=stream)
-        api.dsa_indexer_decode(q, cache, w, seq_lens, q_lens, k, k_base=k_base, out_idx=out_idx,
-                               out_score=out_score, stream=stream)
+    hx = Harness(wl, inp, dev, stream)
 
     # uncaptured warm-up (also plans the batch once)
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
-            step()
+            hx.step()
     api.dsa_check_device_errors(stream)
 
     # capture G steps, each with its own kernel-timing events
@@ -291,14 +370,13 @@ def run_ours(args):
     with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
         for g in range(G):
             api.dsa_set_profile_events(*ev[g])
-            step()
+            hx.step()
         api.dsa_set_profile_events(None, None, None)
     launches_per_step = (api.dsa_kernel_launch_count() - n0) / G
     replays = max(1, args.steps // G)
     K = replays * G
     with torch.cuda.stream(stream):
-        for _ in range(2):
-            graph.replay()
+        graph.replay()
     stream.synchronize()
     api.dsa_check_device_errors(stream)
 
@@ -337,24 +415,32 @@ def run_ours(args):
     pairs_step = wl.pairs * world
     value = pairs_step / (ms_step * 1e-3)
 
-    # end to end through the host-buffer entry point: upload inputs, run, read results back
-    q_h = torch.from_numpy(inp["q_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
-    w_h = torch.from_numpy(inp["w"]).pin_memory()
-    k_h = torch.from_numpy(k_new_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    rows_h = torch.from_numpy(k_base + L - 1).pin_memory()
-    bufs = {}
-    for _ in range(5):
-        api.dsa_indexer_decode_from_host(q_h, w_h, k_h, rows_h, cache, seq_lens, q_lens, k, k_base=k_base,
-                                         dev_bufs=bufs, stream=stream)
+    # end to end from pinned host buffers: upload the step's inputs, run, read the result back
+    k_h, q_h, w_h = hx.k_step_host.pin_memory(), hx.q_src_host.pin_memory(), hx.w_host.pin_memory()
+    k_d, q_d, w_d = torch.empty_like(hx.k_step), torch.empty_like(hx.q_src), torch.empty_like(hx.w)
+    oi_h = torch.empty(hx.out_idx.shape, dtype=torch.int32, pin_memory=True)
+    os_h = torch.empty(hx.out_score.shape, dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            k_d.copy_(k_h, non_blocking=True)
+            q_d.copy_(q_h, non_blocking=True)
+            w_d.copy_(w_h, non_blocking=True)
+            hx.step(k_step=k_d, q_src=q_d, w=w_d)
+            oi_h.copy_(hx.out_idx, non_blocking=True)
+            os_h.copy_(hx.out_score, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    E = max(1, args.e2e_steps if hx.decode else min(args.e2e_steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    E = max(1, args.e2e_steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
     for _ in range(E):
-        api.dsa_indexer_decode_from_host(q_h, w_h, k_h, rows_h, cache, seq_lens, q_lens, k, k_base=k_base,
-                                         dev_bufs=bufs, stream=stream)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / E
@@ -362,17 +448,30 @@ def run_ours(args):
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, w_h, k_h, rows_h))
-    d2h = S * k * (4 + 4)
+    h2d = sum(t.numel() * t.element_size() for t in (k_h, q_h, w_h))
+    d2h = sum(t.numel() * t.element_size() for t in (oi_h, os_h))
 
-    # roofline of the dominant kernel (decode logits): algorithmic bytes it must read
-    alg_bytes = S * L * d * 2 + S * H * d * 2 + S * H * 4
-    achieved = alg_bytes / (logits_ms * 1e-3) / 1e9
-    peak, peak_kind = peaks()
-    traffic = profiled_traffic()
+    # roofline of the dominant kernel (the logits kernel)
+    pk = peaks()
+    if hx.decode:
+        alg = hx.logits_bytes()
+        achieved = alg / (logits_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "traffic": profiled_traffic() if args.workload == "decode" else None,
+                "peak_source": f"{pk['kind']} hbm_gbs", "alg_bytes_per_launch": alg}
+    else:
+        alg = hx.logits_flops()
+        achieved = alg / (logits_ms * 1e-3) / 1e12
+        peak = pk["fp8_sustained"] if hx.fp8 else pk["bf16_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": (f"{pk['kind']} bf16_tflops_sustained" + (" x 2 (FP8/bf16 nominal ratio)" if hx.fp8 else "")),
+                "alg_flops_per_launch": alg,
+                "frac_of_burst_peak": achieved / (pk["fp8_burst"] if hx.fp8 else pk["bf16_burst"])}
+    roof.update({"kernel": f"logits ({wl.kind}, {wl.dtype})", "kernel_ms": logits_ms})
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "decode":
         cpu = oracle_sample(wl, inp, args.cpu_seconds)
 
     if world > 1:
@@ -381,15 +480,13 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "pairs_per_step_per_gpu": wl.pairs,
-                       "l2": "inputs larger than L2 (268 MB bf16 K cache per GPU), no flush",
-                       "step": "kcache_append + decode (logits + top-k), CUDA graph of %d steps" % G,
+            "dtype": "fp8_e4m3" if hx.fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "pairs_per_step_per_gpu": wl.pairs,
+                       "l2": "inputs larger than L2 (126 MB), no flush",
+                       "step": ("kcache_append + " + ("quantise q + " if hx.fp8 else "") +
+                                ("decode" if hx.decode else "prefill") + " (logits + top-k), CUDA graph of %d steps" % G),
                        "parallelism": f"{world} independent ranks (sequences sharded)"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "logits (decode, bf16)", "kernel_ms": logits_ms,
-                         "peak_source": f"{peak_kind} hbm_gbs", "alg_bytes_per_launch": alg_bytes},
+            "roofline": roof,
             "kernels_ms": {"logits": logits_ms, "topk": topk_ms},
             "cpu_baseline": cpu,
             "e2e": {"value": pairs_step / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -100,13 +100,15 @@ def dsa_indexer_kcache_append(cache: IndexerKCache, k_new: torch.Tensor, dst_row
                                                 k_new.shape[0], _stream(stream)))
 
 
-def dsa_quantize_rows_fp8(src: torch.Tensor, stream=None):
+def dsa_quantize_rows_fp8(src: torch.Tensor, dst=None, scale=None, stream=None):
     """Per-row FP8 E4M3 quantisation of ``src`` [rows, ...] (bf16 / fp32): returns (codes uint8, scale fp32 [rows])."""
-    _require_cuda(src)
+    _require_cuda(src, dst, scale)
     rows = src.shape[0]
     row_len = src.numel() // max(rows, 1) if rows else 0
-    dst = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
-    scale = torch.empty(rows, dtype=torch.float32, device=src.device)
+    if dst is None:
+        dst = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    if scale is None:
+        scale = torch.empty(rows, dtype=torch.float32, device=src.device)
     check(_lib.load().dsa_quantize_rows_fp8(_ptr(src), _dtype_code(src), rows, row_len, _ptr(dst), _ptr(scale),
                                             _stream(stream)))
     return dst, scale

@@ -32,6 +32,8 @@ namespace dsa {
 
 namespace {
 
+constexpr int kScalePrefetch = 4;   // tiles of FP8 key scales in flight ahead of the epilogue
+
 template <int H_, int D_, bool FP8_, int TPA_, int NG_, int NE_, int STAGES_>
 struct Cfg {
   static constexpr int H = H_, D = D_, TPA = TPA_, NG = NG_, NE = NE_, STAGES = STAGES_;
@@ -57,6 +59,9 @@ struct Cfg {
   static_assert(Q_BLOCK_BYTES % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
   static constexpr int Q_BYTES = NG * KB * Q_BLOCK_BYTES;
   static constexpr int THREADS = (2 + NE) * 32;
+  // queries whose TMEM loads share one tcgen05.wait::ld: 2 when 4 epilogue warps leave
+  // room for 2 x H live registers per thread, else 1
+  static constexpr int QB = NE == 4 ? 2 : 1;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + STAGES * K_TILE_BYTES;
@@ -91,21 +96,27 @@ __device__ __forceinline__ void issue_umma(uint32_t d_tmem, uint32_t k_stage_add
   }
 }
 
-// sum_h w[h] * max(x[h], 0) over 32 TMEM columns starting at column `col`.
-__device__ __forceinline__ float relu_dot32(uint32_t taddr, const float* __restrict__ w) {
-  uint32_t r[32];
-  tmem_ld_32x32b_x32(taddr, r);
-  tmem_ld_wait();
-  float s0 = 0.f, s1 = 0.f;
+// a0, a1 += w[h] * max(x[h], 0) over 32 accumulator columns already loaded into r,
+// with packed fp32x2 FMAs: 1.5 issue slots per element.
+__device__ __forceinline__ void relu_wsum32(const uint32_t (&r)[32], const float* __restrict__ w, float2& a0,
+                                            float2& a1) {
 #pragma unroll
   for (int h = 0; h < 32; h += 4) {
     const float4 wv = *reinterpret_cast<const float4*>(w + h);
-    s0 = fmaf(wv.x, fmaxf(__uint_as_float(r[h + 0]), 0.f), s0);
-    s1 = fmaf(wv.y, fmaxf(__uint_as_float(r[h + 1]), 0.f), s1);
-    s0 = fmaf(wv.z, fmaxf(__uint_as_float(r[h + 2]), 0.f), s0);
-    s1 = fmaf(wv.w, fmaxf(__uint_as_float(r[h + 3]), 0.f), s1);
+    const float2 x01 = make_float2(fmaxf(__uint_as_float(r[h]), 0.f), fmaxf(__uint_as_float(r[h + 1]), 0.f));
+    const float2 x23 = make_float2(fmaxf(__uint_as_float(r[h + 2]), 0.f), fmaxf(__uint_as_float(r[h + 3]), 0.f));
+    a0 = __ffma2_rn(make_float2(wv.x, wv.y), x01, a0);
+    a1 = __ffma2_rn(make_float2(wv.z, wv.w), x23, a1);
   }
-  return s0 + s1;
+}
+
+// The same over one query's CPT*32 columns.
+template <int CPT>
+__device__ __forceinline__ float relu_wsum(const uint32_t (&r)[CPT][32], const float* __restrict__ w) {
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) relu_wsum32(r[c], w + c * 32, a0, a1);
+  return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
 template <class C>
@@ -251,29 +262,76 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
       __syncwarp();
       const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
       const int pos_last = wi.pos0 + wi.n_tok - 1;
+      // FP8 key scales are loaded kScalePrefetch tiles ahead of use, so the per-tile
+      // global-memory latency overlaps the epilogues of the tiles in between.
+      constexpr int PF = kScalePrefetch;
+      float ks_ring[PF];
+      auto load_scale = [&](int kt) -> float {
+        const int key = kt * C::BM + sub * 32 + lane;
+        const int64_t krow = wi.k_row0 + key;
+        return (kt < wi.kt_end && key <= pos_last && krow < args.k_capacity) ? __ldg(args.k_scale + krow) : 0.f;
+      };
+      if constexpr (C::FP8) {
+#pragma unroll
+        for (int i = 0; i < PF; ++i) ks_ring[i] = load_scale(wi.kt_begin + i);
+      }
       for (int kt = wi.kt_begin; kt < wi.kt_end && ok; ++kt) {
         const int key0 = kt * C::BM;                      // first key of the tile
         const int key = key0 + sub * 32 + lane;           // this thread's key (its TMEM lane)
         float kscale = 1.f;
         if constexpr (C::FP8) {
-          const int64_t krow = wi.k_row0 + key;
-          kscale = (key <= pos_last && krow < args.k_capacity) ? __ldg(args.k_scale + krow) : 0.f;
+          kscale = ks_ring[0];
+#pragma unroll
+          for (int i = 0; i + 1 < PF; ++i) ks_ring[i] = ks_ring[i + 1];
+          ks_ring[PF - 1] = load_scale(kt + PF);
         }
         for (int g = 0; g < groups; ++g, ++acc_iter) {
           const int b = acc_iter % C::NBUF;
-          if (!mbar_wait(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait<true>(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::ACC_COLS;
           const int j_lo = g * C::TPA;
           const int j_hi = min(j_lo + C::TPA, wi.n_tok);
-          if constexpr (C::H >= 32) {
+          if constexpr (C::H >= 32 && C::NE >= 16) {
+            // many epilogue warps: one 32-column chunk in registers at a time
+            constexpr int CPT = C::H / 32;
             for (int j = j_lo + part; j < j_hi; j += SPLIT) {
-              if (key0 > wi.pos0 + j) continue;           // whole tile after this query: nothing to store
-              float acc = 0.f;
+              if (key0 > wi.pos0 + j) continue;                        // the tile is after this query
+              float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-              for (int c = 0; c < C::H / 32; ++c)
-                acc += relu_dot32(tbase + (j - j_lo) * C::H + c * 32, wq + j * C::H + c * 32);
-              if (key <= wi.pos0 + j) args.scores[rowoff[j] + key] = acc * kscale;
+              for (int c = 0; c < CPT; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tbase + (j - j_lo) * C::H + c * 32, r);
+                tmem_ld_wait();
+                relu_wsum32(r, wq + j * C::H + c * 32, a0, a1);
+              }
+              if (key <= wi.pos0 + j) args.scores[rowoff[j] + key] = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+            }
+          } else if constexpr (C::H >= 32) {
+            // QB queries per pass: their loads are in flight behind one tcgen05.wait::ld
+            constexpr int CPT = C::H / 32;
+            for (int j0 = j_lo + part; j0 < j_hi; j0 += C::QB * SPLIT) {
+              uint32_t r[C::QB][CPT][32];
+              bool live[C::QB];
+              bool any = false;
+#pragma unroll
+              for (int u = 0; u < C::QB; ++u) {
+                const int j = j0 + u * SPLIT;
+                live[u] = j < j_hi && key0 <= wi.pos0 + j;             // warp-uniform
+                any |= live[u];
+                if (live[u]) {
+#pragma unroll
+                  for (int c = 0; c < CPT; ++c) tmem_ld_32x32b_x32(tbase + (j - j_lo) * C::H + c * 32, r[u][c]);
+                }
+              }
+              if (!any) continue;                                      // the tile is after these queries
+              tmem_ld_wait();
+#pragma unroll
+              for (int u = 0; u < C::QB; ++u) {
+                const int j = j0 + u * SPLIT;
+                if (live[u] && key <= wi.pos0 + j)
+                  args.scores[rowoff[j] + key] = relu_wsum<CPT>(r[u], wq + j * C::H) * kscale;
+              }
             }
           } else {
             // H < 32: one 32-column load holds 32/H queries
@@ -334,13 +392,13 @@ cudaError_t launch_cfg(const LogitsLaunch& L, const CUtensorMap& tk, const CUten
 // indexer shape ("Study MLA Indexer", 关键参数); H=4/d=64 serves small models.
 //                                  H   D   FP8   TPA NG NE STAGES
 using CfgPrefillBf16   = Cfg<64, 128, false, 4, 2, 8, 2>;
-using CfgPrefillFp8    = Cfg<64, 128, true,  4, 2, 8, 4>;
+using CfgPrefillFp8    = Cfg<64, 128, true,  4, 2, 16, 4>;
 using CfgDecode1Bf16   = Cfg<64, 128, false, 1, 1, 4, 6>;
-using CfgDecode2Bf16   = Cfg<64, 128, false, 2, 1, 4, 5>;
-using CfgDecode4Bf16   = Cfg<64, 128, false, 4, 1, 4, 4>;
+using CfgDecode2Bf16   = Cfg<64, 128, false, 2, 1, 8, 5>;
+using CfgDecode4Bf16   = Cfg<64, 128, false, 4, 1, 8, 4>;
 using CfgDecode1Fp8    = Cfg<64, 128, true,  1, 1, 4, 10>;
-using CfgDecode2Fp8    = Cfg<64, 128, true,  2, 1, 4, 10>;
-using CfgDecode4Fp8    = Cfg<64, 128, true,  4, 1, 4, 10>;
+using CfgDecode2Fp8    = Cfg<64, 128, true,  2, 1, 8, 10>;
+using CfgDecode4Fp8    = Cfg<64, 128, true,  4, 1, 8, 10>;
 using CfgPrefillSmallH = Cfg<4,  64,  false, 64, 1, 4, 4>;
 
 template <class... Cs>

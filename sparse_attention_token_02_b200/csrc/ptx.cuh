@@ -12,6 +12,9 @@ namespace dsa {
 // A wait that has not completed after this many SM cycles (about a second at
 // 1.9 GHz) is abandoned: the kernel records DSA_DEVERR_TIMEOUT and winds down.
 constexpr long long kWaitLimitCycles = 2000000000LL;
+// Upper bound of one sleep inside mbarrier.try_wait (the thread wakes as soon as the
+// phase completes); far below the limit above, so the limit is still checked often.
+constexpr uint32_t kTryWaitSuspendNs = 1000000u;
 
 // Records the first device fault of a call: err[0] = code, err[1] = info.
 __device__ __forceinline__ void record_error(int* err, int code, int info) {
@@ -41,25 +44,41 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// One probe of the phase.  With kSleep the thread may sleep inside the probe (up to
+// the hint, in ns) until the phase completes, so many waiting warps do not spin on
+// the issue slots; without it the probe returns at once (lowest wake-up latency, for
+// the single-lane producer and MMA roles).
+template <bool kSleep>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
+  if constexpr (kSleep) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kTryWaitSuspendNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+  }
   return done != 0;
 }
 
 // Waits for the phase with the given parity to complete.  Returns false if the
 // wait ran past kWaitLimitCycles or another role raised *abort (volatile smem).
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait<kSleep>(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kSleep>(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitLimitCycles) {
       *abort = 1;

@@ -297,3 +297,37 @@ def test_full_ragged_decode_fp8_sampled_sequences():
     seqs = [int(order[0]), int(order[-1]), int(order[len(order) // 2])]
     rows = sorted(2 * b + j for b in seqs for j in (0, 1))
     _check(up, idx, sc, rows)
+
+
+# ----------------------------------------------------------------------------- CUDA graphs
+
+def test_graph_capture_replay_equals_eager_and_unplanned_capture_is_refused():
+    wl = W.scaled(W.decode(), seq_lens=(3000, 2500, 40), q_lens=(1, 1, 1), seed=31)
+    up = Uploaded(wl)
+    s = torch.cuda.Stream()
+    out_i = torch.empty(3, wl.top_k, dtype=torch.int32, device="cuda")
+    out_s = torch.empty(3, wl.top_k, dtype=torch.float32, device="cuda")
+    run = lambda: api.dsa_indexer_decode(up.q, up.cache, up.w, wl.seq_lens, wl.q_lens, wl.top_k, k_base=up.k_base,
+                                         out_idx=out_i, out_score=out_s, stream=s)
+    with torch.cuda.stream(s):
+        run()
+    s.synchronize()
+    eager_i, eager_s = out_i.clone(), out_s.clone()
+    out_i.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+        run()
+        # a batch this stream has not run uncaptured cannot be planned during capture
+        with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+            api.dsa_indexer_decode(up.q[:2], up.cache, up.w[:2], (3000, 2500), (1, 1), wl.top_k,
+                                   k_base=up.k_base[:2], stream=s)
+    for _ in range(3):
+        g.replay()
+    s.synchronize()
+    # the order inside a row is unspecified: compare each row's (index, score) pairs sorted by index
+    for a_i, a_s, b_i, b_s in zip(out_i.cpu().numpy(), out_s.cpu().numpy(), eager_i.cpu().numpy(),
+                                  eager_s.cpu().numpy()):
+        oa, ob = np.argsort(a_i), np.argsort(b_i)
+        assert np.array_equal(a_i[oa], b_i[ob]) and np.array_equal(a_s[oa], b_s[ob])
+    del g
+    api.dsa_check_device_errors(s)
