@@ -61,6 +61,24 @@ def parse():
     return ap.parse_args()
 
 
+# ----------------------------------------------------------------------------- multi-rank aggregation
+
+def max_over_ranks(x: float, dist=None) -> float:
+    """The slowest rank's value (the job's time); x itself without a process group."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(pairs_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the pairs every rank scored and selected per second of the slowest rank."""
+    return pairs_per_rank * world / (ms_per_step * 1e-3)
+
+
 # ----------------------------------------------------------------------------- workload
 
 def workload(rank: int, name: str = "decode"):
@@ -407,13 +425,10 @@ def run_ours(args):
     logits_ms = statistics.mean(ev[g][0].elapsed_time(ev[g][1]) for g in range(G))
     topk_ms = statistics.mean(ev[g][1].elapsed_time(ev[g][2]) for g in range(G))
     api.dsa_check_device_errors(stream)
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dist if world > 1 else None)
     ms_step = ms_total / K
     pairs_step = wl.pairs * world
-    value = pairs_step / (ms_step * 1e-3)
+    value = job_value(wl.pairs, world, ms_step)
 
     # end to end from pinned host buffers: upload the step's inputs, run, read the result back
     k_h, q_h, w_h = hx.k_step_host.pin_memory(), hx.q_src_host.pin_memory(), hx.w_host.pin_memory()
@@ -443,11 +458,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / E
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, dist if world > 1 else None)
     h2d = sum(t.numel() * t.element_size() for t in (k_h, q_h, w_h))
     d2h = sum(t.numel() * t.element_size() for t in (oi_h, os_h))
 

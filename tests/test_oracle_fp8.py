@@ -83,3 +83,11 @@ def test_quantize_rows_scale_and_error_bound():
     bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scale[:, None]) * (1 + 1e-6)
     assert np.all(err <= bound)
     assert E4M3_MAX == 448.0
+
+
+def test_bf16_bits_decode_matches_torch():
+    from oracle import bf16_bits_to_f64
+    x = torch.randn(50000, dtype=torch.float32) * 100
+    b = x.to(torch.bfloat16)
+    bits = b.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf16_bits_to_f64(bits), b.to(torch.float64).numpy())
