@@ -10,7 +10,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdsa_indexer.so")
+# DSA_INDEXER_LIB may name another build of the same library (e.g. a tuning variant)
+LIB_PATH = os.environ.get("DSA_INDEXER_LIB") or os.path.join(_HERE, "libdsa_indexer.so")
 
 DSA_BF16, DSA_FP8_E4M3, DSA_F32 = 0, 1, 2
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_ALLOC",

@@ -50,14 +50,17 @@ def _stale(target: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(jobs: int = 8, verbose: bool = False, extra: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(jobs: int = 8, verbose: bool = False, extra: list[str] | None = None, out_dir: str | None = None) -> str:
+    """Build the library; `extra` nvcc flags and `out_dir` (objects and .so) serve tuning builds."""
+    build_dir = os.path.join(out_dir, "_build") if out_dir else BUILD
+    lib_path = os.path.join(out_dir, "libdsa_indexer.so") if out_dir else LIB
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = _headers()
     cmds = []
     objs = []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if _stale(obj, [src] + headers):
             cmds.append([nvcc(), *ARCH, *CFLAGS, *(extra or []), "-c", src, "-o", obj])
@@ -73,9 +76,9 @@ def build(jobs: int = 8, verbose: bool = False, extra: list[str] | None = None) 
 
     with cf.ThreadPoolExecutor(max_workers=max(1, jobs)) as ex:
         list(ex.map(run, cmds))
-    if cmds or _stale(LIB, objs):
-        run([nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", LIB, *objs])
-    return LIB
+    if cmds or _stale(lib_path, objs):
+        run([nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", lib_path, *objs])
+    return lib_path
 
 
 def main(argv=None) -> int:

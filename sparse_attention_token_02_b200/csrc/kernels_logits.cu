@@ -33,10 +33,20 @@ namespace dsa {
 namespace {
 
 constexpr int kScalePrefetch = 4;   // tiles of FP8 key scales in flight ahead of the epilogue
+#ifndef DSA_TMEM_X64
+#define DSA_TMEM_X64 0                  // one 64-column TMEM load per query instead of two
+#endif
 
-template <int H_, int D_, bool FP8_, int TPA_, int NG_, int NE_, int STAGES_>
+template <int H_, int D_, bool FP8_, int TPA_, int NG_, int NE_, int STAGES_, int EG_ = 1>
 struct Cfg {
   static constexpr int H = H_, D = D_, TPA = TPA_, NG = NG_, NE = NE_, STAGES = STAGES_;
+  // Epilogue warps form EG groups; group g drains accumulators g, g+EG, ... so EG
+  // accumulators are drained at once.  Inside a group, the SPLIT warps that share a TMEM
+  // subpartition split the accumulator's queries.
+  static constexpr int EG = EG_;
+  static constexpr int NEG = NE / EG;
+  static constexpr int SPLIT = NEG / 4;
+  static_assert(NEG % 4 == 0 && NE % EG == 0, "epilogue groups cover the 4 TMEM subpartitions");
   static constexpr bool FP8 = FP8_;
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int ROW_BYTES = D * ESZ;
@@ -59,9 +69,20 @@ struct Cfg {
   static_assert(Q_BLOCK_BYTES % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
   static constexpr int Q_BYTES = NG * KB * Q_BLOCK_BYTES;
   static constexpr int THREADS = (2 + NE) * 32;
-  // queries whose TMEM loads share one tcgen05.wait::ld: 2 when 4 epilogue warps leave
-  // room for 2 x H live registers per thread, else 1
-  static constexpr int QB = NE == 4 ? 2 : 1;
+  static_assert(EG <= NBUF, "each epilogue group needs its own accumulator buffer");
+  // Register budget per thread decides how many TMEM columns stay live: 2 queries (192
+  // threads, up to 255 registers), 1 query (up to 168), one 32-column chunk (fewer).
+  static constexpr int QB = THREADS <= 256 ? 2 : 1;
+  static constexpr bool CHUNKED = THREADS > 384;
+  // every epilogue warp owns exactly one query of the work item: its head weights stay
+  // in registers for the whole item
+  static constexpr bool ONE_QUERY_PER_WARP = (NG == 1) && (TPA == SPLIT) && (H == 64) && !CHUNKED;
+  // epilogue warps sleep inside their accumulator waits only when there are so many of
+  // them that spinning would take issue slots from the ones computing
+  static constexpr bool EPI_SLEEP = NE >= 16;
+  // the producer and MMA lanes sleep in their waits when the epilogue, not their
+  // latency, sets the pace (prefill): then they leave the issue slots to the epilogue
+  static constexpr bool PIPE_SLEEP = NG > 1;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + STAGES * K_TILE_BYTES;
@@ -110,6 +131,18 @@ __device__ __forceinline__ void relu_wsum32(const uint32_t (&r)[32], const float
   }
 }
 
+// The same with the 32 weights already in registers.
+__device__ __forceinline__ void relu_wsum32_reg(const uint32_t (&r)[32], const float2 (&w)[16], float2& a0,
+                                                float2& a1) {
+#pragma unroll
+  for (int h = 0; h < 32; h += 4) {
+    const float2 x01 = make_float2(fmaxf(__uint_as_float(r[h]), 0.f), fmaxf(__uint_as_float(r[h + 1]), 0.f));
+    const float2 x23 = make_float2(fmaxf(__uint_as_float(r[h + 2]), 0.f), fmaxf(__uint_as_float(r[h + 3]), 0.f));
+    a0 = __ffma2_rn(w[h / 2], x01, a0);
+    a1 = __ffma2_rn(w[h / 2 + 1], x23, a1);
+  }
+}
+
 // The same over one query's CPT*32 columns.
 template <int CPT>
 __device__ __forceinline__ float relu_wsum(const uint32_t (&r)[CPT][32], const float* __restrict__ w) {
@@ -119,12 +152,26 @@ __device__ __forceinline__ float relu_wsum(const uint32_t (&r)[CPT][32], const f
   return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
+#ifdef DSA_PIPE_STATS
+// Tuning builds only: cycles each role spends waiting, summed over CTAs.
+// 0 producer waits for a free K stage, 1 MMA waits for a loaded K tile, 2 MMA waits for a
+// free accumulator, 3 epilogue (first warp) waits for a finished accumulator, 4 epilogue
+// (first warp) compute, 5 CTA cycles, 6 producer waits for the Q buffer, 7 MMA waits for Q.
+__device__ unsigned long long g_pipe_stats[8];
+#define DSA_TIMED(slot, expr) ([&]() { const long long t0_ = clock64(); const bool r_ = (expr); \
+                                        st_[slot] += clock64() - t0_; return r_; }())
+#else
+#define DSA_TIMED(slot, expr) (expr)
+#endif
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
 logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
               const LogitsArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the __shared__ array by an offset so that the
+  // compiler keeps the shared address space (ld.shared / st.shared with 32-bit addresses)
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + C::STAGES;
@@ -138,8 +185,10 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int item_begin = args.cta_items[blockIdx.x];
-  const int item_end = args.cta_items[blockIdx.x + 1];
+#ifdef DSA_PIPE_STATS
+  long long st_[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const long long t_start_ = clock64();
+#endif
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -150,7 +199,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
     mbar_init(q_empty, 1);
     for (int b = 0; b < C::NBUF; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], C::NE);
+      mbar_init(&acc_empty[b], C::NEG);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -167,6 +216,12 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t smem_base = smem_addr(smem);
+  // The prologue above overlaps the previous kernel; its outputs (appended keys, quantised
+  // queries) are read only after this point.  The next kernel may start its own prologue.
+  grid_dependency_wait();
+  launch_dependents();
+  const int item_begin = args.cta_items[blockIdx.x];
+  const int item_end = args.cta_items[blockIdx.x + 1];
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -177,7 +232,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
       bool ok = true;
       for (int it = item_begin; it < item_end && ok; ++it) {
         const LogitsItem wi = args.items[it];
-        if (!mbar_wait(q_empty, (item_iter & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!DSA_TIMED(6, mbar_wait<C::PIPE_SLEEP>(q_empty, (item_iter & 1) ^ 1, abort_flag))) { ok = false; break; }
         mbar_arrive_expect_tx(q_full, C::Q_BYTES);
         for (int g = 0; g < C::NG; ++g)
           for (int kb = 0; kb < C::KB; ++kb)
@@ -186,7 +241,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
         ++item_iter;
         for (int kt = wi.kt_begin; kt < wi.kt_end; ++kt, ++k_iter) {
           const int s = k_iter % C::STAGES;
-          if (!mbar_wait(&k_empty[s], ((k_iter / C::STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (!DSA_TIMED(0, mbar_wait<C::PIPE_SLEEP>(&k_empty[s], ((k_iter / C::STAGES) & 1) ^ 1, abort_flag))) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[s], C::K_TILE_BYTES);
           const int32_t y = static_cast<int32_t>(wi.k_row0 + static_cast<int64_t>(kt) * C::BM);
           for (int kb = 0; kb < C::KB; ++kb)
@@ -215,15 +270,15 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
       for (int it = item_begin; it < item_end && ok; ++it) {
         const LogitsItem wi = args.items[it];
         const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
-        if (!mbar_wait(q_full, item_iter & 1, abort_flag)) { ok = false; break; }
+        if (!DSA_TIMED(7, mbar_wait<C::PIPE_SLEEP>(q_full, item_iter & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
         for (int kt = wi.kt_begin; kt < wi.kt_end && ok; ++kt, ++k_iter) {
           const int s = k_iter % C::STAGES;
-          if (!mbar_wait(&k_full[s], (k_iter / C::STAGES) & 1, abort_flag)) { ok = false; break; }
+          if (!DSA_TIMED(1, mbar_wait<C::PIPE_SLEEP>(&k_full[s], (k_iter / C::STAGES) & 1, abort_flag))) { ok = false; break; }
           tc_fence_after();
           for (int g = 0; g < groups; ++g, ++acc_iter) {
             const int b = acc_iter % C::NBUF;
-            if (!mbar_wait(&acc_empty[b], ((acc_iter / C::NBUF) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!DSA_TIMED(2, mbar_wait<C::PIPE_SLEEP>(&acc_empty[b], ((acc_iter / C::NBUF) & 1) ^ 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
             issue_umma<C>(tmem_base + b * C::ACC_COLS, smem_base + C::OFF_K + s * C::K_TILE_BYTES,
                           smem_base + C::OFF_Q + g * C::KB * C::Q_BLOCK_BYTES);
@@ -243,8 +298,9 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
     // ------------------------------------------------------------------ epilogue
     const int ew = warp - 2;                  // 0 .. NE-1
     const int sub = warp & 3;                 // TMEM subpartition this warp may access
-    constexpr int SPLIT = C::NE / 4;          // warps sharing one subpartition
-    const int part = ew / 4;                  // which share of the queries this warp takes
+    constexpr int SPLIT = C::SPLIT;           // warps of a group sharing one subpartition
+    const int grp = ew / C::NEG;              // accumulators grp, grp+EG, ... are this warp's
+    const int part = (ew % C::NEG) / 4;       // which share of an accumulator's queries
     float* wq = reinterpret_cast<float*>(smem + C::OFF_W) + ew * C::W_WARP_FLOATS;
     int64_t* rowoff = reinterpret_cast<int64_t*>(smem + C::OFF_ROW) + ew * C::NT;
     uint32_t acc_iter = 0;
@@ -260,6 +316,15 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
       }
       for (int j = lane; j < wi.n_tok; j += 32) rowoff[j] = args.row_off[wi.q_row0 + j];
       __syncwarp();
+      float2 wr_lo[16], wr_hi[16];                // this warp's query's w' (ONE_QUERY_PER_WARP)
+      if constexpr (C::ONE_QUERY_PER_WARP) {
+        const int j = part < wi.n_tok ? part : 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          wr_lo[i] = *reinterpret_cast<const float2*>(wq + j * 64 + 2 * i);
+          wr_hi[i] = *reinterpret_cast<const float2*>(wq + j * 64 + 32 + 2 * i);
+        }
+      }
       const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
       const int pos_last = wi.pos0 + wi.n_tok - 1;
       // FP8 key scales are loaded kScalePrefetch tiles ahead of use, so the per-tile
@@ -286,13 +351,37 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
           ks_ring[PF - 1] = load_scale(kt + PF);
         }
         for (int g = 0; g < groups; ++g, ++acc_iter) {
+          if (C::EG > 1 && static_cast<int>(acc_iter % C::EG) != grp) continue;   // another group's
           const int b = acc_iter % C::NBUF;
-          if (!mbar_wait<true>(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag)) { ok = false; break; }
+          if (!DSA_TIMED(3, mbar_wait<C::EPI_SLEEP>(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag))) { ok = false; break; }
+#ifdef DSA_PIPE_STATS
+          const long long tc0_ = clock64();
+#endif
           tc_fence_after();
           const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::ACC_COLS;
           const int j_lo = g * C::TPA;
           const int j_hi = min(j_lo + C::TPA, wi.n_tok);
-          if constexpr (C::H >= 32 && C::NE >= 16) {
+          if constexpr (C::ONE_QUERY_PER_WARP) {
+            const int j = part;                                        // this warp's query
+            if (j < wi.n_tok && key0 <= wi.pos0 + j) {                 // warp-uniform
+              float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#if DSA_TMEM_X64
+              uint32_t r[64];
+              tmem_ld_32x32b_x64(tbase + j * 64, r);
+              tmem_ld_wait();
+              relu_wsum32_reg(*reinterpret_cast<uint32_t(*)[32]>(r), wr_lo, a0, a1);
+              relu_wsum32_reg(*reinterpret_cast<uint32_t(*)[32]>(r + 32), wr_hi, a0, a1);
+#else
+              uint32_t r0[32], r1[32];
+              tmem_ld_32x32b_x32(tbase + j * 64, r0);
+              tmem_ld_32x32b_x32(tbase + j * 64 + 32, r1);
+              tmem_ld_wait();
+              relu_wsum32_reg(r0, wr_lo, a0, a1);
+              relu_wsum32_reg(r1, wr_hi, a0, a1);
+#endif
+              if (key <= wi.pos0 + j) args.scores[rowoff[j] + key] = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+            }
+          } else if constexpr (C::H >= 32 && C::CHUNKED) {
             // many epilogue warps: one 32-column chunk in registers at a time
             constexpr int CPT = C::H / 32;
             for (int j = j_lo + part; j < j_hi; j += SPLIT) {
@@ -357,6 +446,9 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
           }
           tc_fence_before();
           __syncwarp();
+#ifdef DSA_PIPE_STATS
+          st_[4] += clock64() - tc0_;
+#endif
           if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
       }
@@ -371,6 +463,22 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
   if (threadIdx.x == 0 && *abort_flag) record_error(args.err, DSA_DEVERR_TIMEOUT, blockIdx.x);
+#ifdef DSA_PIPE_STATS
+  if (threadIdx.x == 0) {                     // producer lane
+    atomicAdd(&g_pipe_stats[0], st_[0]);
+    atomicAdd(&g_pipe_stats[6], st_[6]);
+    atomicAdd(&g_pipe_stats[5], clock64() - t_start_);
+  }
+  if (threadIdx.x == 32) {                    // MMA lane
+    atomicAdd(&g_pipe_stats[1], st_[1]);
+    atomicAdd(&g_pipe_stats[2], st_[2]);
+    atomicAdd(&g_pipe_stats[7], st_[7]);
+  }
+  if (threadIdx.x == 64) {                    // first epilogue warp
+    atomicAdd(&g_pipe_stats[3], st_[3]);
+    atomicAdd(&g_pipe_stats[4], st_[4]);
+  }
+#endif
 }
 
 template <class C>
@@ -384,20 +492,61 @@ cudaError_t launch_cfg(const LogitsLaunch& L, const CUtensorMap& tk, const CUten
     if (e != cudaSuccess) return e;
     if (dev < 64) configured |= 1ull << dev;
   }
-  logits_kernel<C><<<L.grid, C::THREADS, C::SMEM_BYTES, L.stream>>>(tk, tq, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(L.grid, 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, logits_kernel<C>, tk, tq, a);
 }
 
 // The configurations this library is built with.  H=64/d=128 is the DeepSeek-V3.2
-// indexer shape ("Study MLA Indexer", 关键参数); H=4/d=64 serves small models.
-//                                  H   D   FP8   TPA NG NE STAGES
-using CfgPrefillBf16   = Cfg<64, 128, false, 4, 2, 8, 2>;
-using CfgPrefillFp8    = Cfg<64, 128, true,  4, 2, 16, 4>;
-using CfgDecode1Bf16   = Cfg<64, 128, false, 1, 1, 4, 6>;
+// indexer shape ("Study MLA Indexer", 关键参数); H=4/d=64 serves small models.  Epilogue
+// warps (NE), pipeline depth (STAGES) and epilogue groups (EG) of each configuration can be
+// overridden at build time, e.g. -DDSA_PF8_STAGES=7, for tuning; the host chooses TPA/NG.
+#ifndef DSA_PB16_NE
+#define DSA_PB16_NE 8
+#endif
+#ifndef DSA_PB16_STAGES
+#define DSA_PB16_STAGES 2
+#endif
+#ifndef DSA_PB16_EG
+#define DSA_PB16_EG 1
+#endif
+#ifndef DSA_PF8_NE
+#define DSA_PF8_NE 16
+#endif
+#ifndef DSA_PF8_STAGES
+#define DSA_PF8_STAGES 4
+#endif
+#ifndef DSA_PF8_EG
+#define DSA_PF8_EG 1
+#endif
+#ifndef DSA_D1B16_NE
+#define DSA_D1B16_NE 4
+#endif
+#ifndef DSA_D1B16_STAGES
+#define DSA_D1B16_STAGES 6
+#endif
+#ifndef DSA_D2F8_NE
+#define DSA_D2F8_NE 8
+#endif
+#ifndef DSA_D2F8_STAGES
+#define DSA_D2F8_STAGES 10
+#endif
+//                                  H   D   FP8   TPA NG NE               STAGES               EG
+using CfgPrefillBf16   = Cfg<64, 128, false, 4, 2, DSA_PB16_NE,  DSA_PB16_STAGES,  DSA_PB16_EG>;
+using CfgPrefillFp8    = Cfg<64, 128, true,  4, 2, DSA_PF8_NE,   DSA_PF8_STAGES,   DSA_PF8_EG>;
+using CfgDecode1Bf16   = Cfg<64, 128, false, 1, 1, DSA_D1B16_NE, DSA_D1B16_STAGES>;
 using CfgDecode2Bf16   = Cfg<64, 128, false, 2, 1, 8, 5>;
 using CfgDecode4Bf16   = Cfg<64, 128, false, 4, 1, 8, 4>;
 using CfgDecode1Fp8    = Cfg<64, 128, true,  1, 1, 4, 10>;
-using CfgDecode2Fp8    = Cfg<64, 128, true,  2, 1, 8, 10>;
+using CfgDecode2Fp8    = Cfg<64, 128, true,  2, 1, DSA_D2F8_NE,  DSA_D2F8_STAGES>;
 using CfgDecode4Fp8    = Cfg<64, 128, true,  4, 1, 8, 10>;
 using CfgPrefillSmallH = Cfg<4,  64,  false, 64, 1, 4, 4>;
 
@@ -408,6 +557,17 @@ static_assert(all_fit<CfgPrefillBf16, CfgPrefillFp8, CfgDecode1Bf16, CfgDecode2B
               "shared memory of a configuration exceeds 227 KB");
 
 }  // namespace
+
+#ifdef DSA_PIPE_STATS
+extern "C" __attribute__((visibility("default"))) int dsa_debug_pipe_stats(unsigned long long* out, int reset) {
+  if (cudaMemcpyFromSymbol(out, g_pipe_stats, sizeof(g_pipe_stats)) != cudaSuccess) return 1;
+  if (reset) {
+    unsigned long long z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (cudaMemcpyToSymbol(g_pipe_stats, z, sizeof(z)) != cudaSuccess) return 1;
+  }
+  return 0;
+}
+#endif
 
 bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng) {
   if (H == 64 && D == 128) {

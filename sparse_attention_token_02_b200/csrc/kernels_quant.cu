@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 quantize_rows_fp8_kernel(const void* __restrict__ src, int src_is_f32, int64_t rows, int32_t row_len,
                          uint8_t* __restrict__ dst, float* __restrict__ scale, const int64_t* __restrict__ dst_rows,
                          int64_t dst_capacity, int* err) {
+  launch_dependents();                        // the indexer kernel may start its prologue
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -83,6 +84,7 @@ quantize_rows_fp8_kernel(const void* __restrict__ src, int src_is_f32, int64_t r
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 append_bf16_kernel(const void* __restrict__ src, int src_is_f32, int64_t rows, int32_t row_len,
                    uint16_t* __restrict__ dst, const int64_t* __restrict__ dst_rows, int64_t dst_capacity, int* err) {
+  launch_dependents();                        // the indexer kernel may start its prologue
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   if (row >= rows) return;

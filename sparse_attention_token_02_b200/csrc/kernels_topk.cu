@@ -151,6 +151,7 @@ topk_kernel(const TopkArgs a) {
     loc_max = 0u;
   }
   __syncthreads();
+  grid_dependency_wait();                     // the scores come from the previous kernel
 
   // ---- load the slice into registers as order-preserving keys (0 = absent); local key range
   uint32_t key[EPT];
@@ -440,6 +441,7 @@ topk_kernel(const TopkArgs a) {
 
 // Rows whose whole causal history fits in top_k: every position, then -1 / -inf.
 __global__ void __launch_bounds__(256) topk_short_kernel(const TopkArgs a) {
+  grid_dependency_wait();                     // the scores come from the previous kernel
   const int row = a.rows[blockIdx.x];
   const int n = a.row_pos[row] + 1;
   const float* src = a.scores + a.row_off[row];
@@ -463,13 +465,15 @@ cudaError_t launch_ept(const TopkArgs& a, int cluster, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kTopkSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   static unsigned long long configured = 0;   // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -498,8 +502,16 @@ cudaError_t launch_topk(const TopkArgs& a, int ept, int cluster, cudaStream_t st
 
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream) {
   if (a.n_rows <= 0) return cudaSuccess;
-  topk_short_kernel<<<a.n_rows, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.n_rows), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_short_kernel, a);
 }
 
 }  // namespace dsa
