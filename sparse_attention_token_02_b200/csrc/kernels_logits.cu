@@ -157,7 +157,7 @@ __device__ __forceinline__ float relu_wsum(const uint32_t (&r)[CPT][32], const f
 // 0 producer waits for a free K stage, 1 MMA waits for a loaded K tile, 2 MMA waits for a
 // free accumulator, 3 epilogue (first warp) waits for a finished accumulator, 4 epilogue
 // (first warp) compute, 5 CTA cycles, 6 producer waits for the Q buffer, 7 MMA waits for Q.
-__device__ unsigned long long g_pipe_stats[8];
+__device__ unsigned long long g_pipe_stats[12];
 #define DSA_TIMED(slot, expr) ([&]() { const long long t0_ = clock64(); const bool r_ = (expr); \
                                         st_[slot] += clock64() - t0_; return r_; }())
 #else
@@ -186,7 +186,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 #ifdef DSA_PIPE_STATS
-  long long st_[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  long long st_[12] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
   const long long t_start_ = clock64();
 #endif
 
@@ -265,6 +265,9 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
+#ifdef DSA_PIPE_STATS
+      st_[10] += clock64() - t_start_;
+#endif
       uint32_t k_iter = 0, acc_iter = 0, item_iter = 0;
       bool ok = true;
       for (int it = item_begin; it < item_end && ok; ++it) {
@@ -280,19 +283,35 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
             const int b = acc_iter % C::NBUF;
             if (!DSA_TIMED(2, mbar_wait<C::PIPE_SLEEP>(&acc_empty[b], ((acc_iter / C::NBUF) & 1) ^ 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
+#ifdef DSA_PIPE_STATS
+            const long long ti0_ = clock64();
+#endif
             issue_umma<C>(tmem_base + b * C::ACC_COLS, smem_base + C::OFF_K + s * C::K_TILE_BYTES,
                           smem_base + C::OFF_Q + g * C::KB * C::Q_BLOCK_BYTES);
+#ifdef DSA_PIPE_STATS
+            const long long ti1_ = clock64();
+            st_[8] += ti1_ - ti0_;
+#endif
             umma_commit(&acc_full[b]);
+#ifdef DSA_PIPE_STATS
+            st_[9] += clock64() - ti1_;
+#endif
           }
           if (ok) umma_commit(&k_empty[s]);
         }
         if (ok) umma_commit(q_empty);
         ++item_iter;
       }
+#ifdef DSA_PIPE_STATS
+      const long long tl_end_ = clock64();
+#endif
       // Let every issued UMMA finish before TMEM is released.
       umma_commit(drain);
       volatile int never = 0;
       mbar_wait(drain, 0, &never);
+#ifdef DSA_PIPE_STATS
+      st_[11] = tl_end_;                      // exit time minus this = drain + final barrier
+#endif
     }
   } else {
     // ------------------------------------------------------------------ epilogue
@@ -470,9 +489,13 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
     atomicAdd(&g_pipe_stats[5], clock64() - t_start_);
   }
   if (threadIdx.x == 32) {                    // MMA lane
+    atomicAdd(&g_pipe_stats[10], st_[10]);
+    atomicAdd(&g_pipe_stats[11], clock64() - st_[11]);
     atomicAdd(&g_pipe_stats[1], st_[1]);
     atomicAdd(&g_pipe_stats[2], st_[2]);
     atomicAdd(&g_pipe_stats[7], st_[7]);
+    atomicAdd(&g_pipe_stats[8], st_[8]);
+    atomicAdd(&g_pipe_stats[9], st_[9]);
   }
   if (threadIdx.x == 64) {                    // first epilogue warp
     atomicAdd(&g_pipe_stats[3], st_[3]);
@@ -562,7 +585,7 @@ static_assert(all_fit<CfgPrefillBf16, CfgPrefillFp8, CfgDecode1Bf16, CfgDecode2B
 extern "C" __attribute__((visibility("default"))) int dsa_debug_pipe_stats(unsigned long long* out, int reset) {
   if (cudaMemcpyFromSymbol(out, g_pipe_stats, sizeof(g_pipe_stats)) != cudaSuccess) return 1;
   if (reset) {
-    unsigned long long z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    unsigned long long z[12] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
     if (cudaMemcpyToSymbol(g_pipe_stats, z, sizeof(z)) != cudaSuccess) return 1;
   }
   return 0;
