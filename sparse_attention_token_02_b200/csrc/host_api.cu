@@ -69,6 +69,7 @@ struct Plan {
   std::vector<int64_t> row_off;
   std::vector<int32_t> row_pos;
   int64_t score_elems = 0;
+  int64_t hist_elems = 0;            // coarse per-row histograms (decode): T_total * kHistBins
   // top-k launches: rows grouped by (ept, cluster); short rows separately
   struct TopkClass {
     int ept, cluster;
@@ -558,12 +559,15 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     else
       plan_prefill_items(v, tpa * ng, ng, g_sms, &np);
     if (mode != Mode::Scores && (st = plan_topk(v, top_k, g_sms, &np)) != DSA_OK) return st;
+    // decode: the logits epilogue bins each row for the top-k (rows are few and long)
+    np.hist_elems = mode == Mode::Decode ? v.total_q * kHistBins : 0;
     const MetaLayout nm = layout_of(np);
     const std::vector<uint8_t> blob = pack(np, nm);
     c->meta_valid = false;
     void* dm = nullptr;
     float* ds = nullptr;
-    if ((st = reserve(c, nm.total, size_t(np.score_elems) * sizeof(float), &dm, &ds)) != DSA_OK) return st;
+    const size_t ws_bytes = align_up(size_t(np.score_elems) * sizeof(float)) + size_t(np.hist_elems) * sizeof(uint32_t);
+    if ((st = reserve(c, nm.total, ws_bytes, &dm, &ds)) != DSA_OK) return st;
     if ((st = stage_upload(c, blob.data(), blob.size(), dm)) != DSA_OK) return st;
     c->plan = std::move(np);
     c->layout = nm;
@@ -577,6 +581,11 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   const MetaLayout& m = c->layout;
   float* d_scores = c->cur_scores;
   char* mb = static_cast<char*>(c->cur_meta);
+  uint32_t* d_hist = p.hist_elems
+      ? reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(d_scores) + align_up(size_t(p.score_elems) * sizeof(float)))
+      : nullptr;
+  if (d_hist)
+    DSA_CUDA_TRY(cudaMemsetAsync(d_hist, 0, size_t(p.hist_elems) * sizeof(uint32_t), stream), "cudaMemsetAsync");
 
   CUtensorMap tk, tq;
   if ((st = encode_rows(&tk, kc->k, fp8, kc->capacity_rows, D, kKeyTile)) != DSA_OK) return st;
@@ -591,6 +600,7 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   la.k_scale = fp8 ? kc->k_scale : nullptr;
   la.k_capacity = kc->capacity_rows;
   la.scores = mode == Mode::Scores ? dense_out : d_scores;
+  la.row_hist = d_hist;
   la.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   la.err = c->d_err;
   LogitsLaunch L{H, D, fp8, tpa, ng, static_cast<int>(p.cta_items.size()) - 1, stream};
@@ -607,6 +617,7 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
 
   TopkArgs ta{};
   ta.scores = d_scores;
+  ta.row_hist = d_hist;
   ta.row_off = la.row_off;
   ta.row_pos = reinterpret_cast<const int32_t*>(mb + m.row_pos);
   ta.top_k = top_k;
@@ -726,7 +737,7 @@ size_t dsa_indexer_workspace_bytes(const dsa_query_t* q, const dsa_batch_t* batc
   const int64_t items = rows + tiles + 4096;   // bound on the number of work items
   const size_t meta = align_up(items * sizeof(LogitsItem)) + align_up((items + 2) * 4) + align_up(rows * 8) +
                       align_up(rows * 4) + align_up(rows * 4);
-  return align_up(meta) + align_up(size_t(elems) * sizeof(float));
+  return align_up(meta) + align_up(size_t(elems) * sizeof(float)) + size_t(rows) * kHistBins * sizeof(uint32_t);
 }
 
 dsa_status_t dsa_set_workspace(void* ptr, size_t bytes, void* stream_v) {

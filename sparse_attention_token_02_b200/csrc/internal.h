@@ -16,6 +16,15 @@ enum : int {
 };
 
 constexpr int kKeyTile = 128;       // keys per UMMA tile (the M dimension)
+// Coarse per-row score histogram built by the decode logits epilogue for the top-k:
+// bins are the top 12 bits of the order-preserving key (sign, exponent, 3 mantissa bits).
+constexpr int kHistShift = 20;
+constexpr int kHistBins = 1 << (32 - kHistShift);
+
+// Order-preserving map of a float to uint32 (larger float -> larger key).
+__host__ __device__ __forceinline__ uint32_t order_key(uint32_t float_bits) {
+  return (float_bits & 0x80000000u) ? ~float_bits : (float_bits | 0x80000000u);
+}
 constexpr int kTopkThreads = 512;   // threads per top-k CTA
 constexpr int kTopkBins = 2048;     // histogram bins per refinement level
 
@@ -41,12 +50,14 @@ struct LogitsArgs {
   const float* k_scale;      // [capacity_rows] (FP8) or nullptr
   int64_t k_capacity;        // rows in the cache (bounds for k_scale reads)
   float* scores;             // workspace
+  uint32_t* row_hist;        // [T_total, kHistBins] zeroed coarse histograms, or nullptr
   float inv_sqrt_d;
   int* err;
 };
 
 struct TopkArgs {
   const float* scores;
+  const uint32_t* row_hist;  // coarse histograms from the logits epilogue, or nullptr
   const int64_t* row_off;
   const int32_t* row_pos;    // [T_total]: position p of each query row (valid keys 0..p)
   const int32_t* rows;       // rows handled by this launch

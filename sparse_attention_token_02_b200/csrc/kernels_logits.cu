@@ -83,6 +83,8 @@ struct Cfg {
   // the producer and MMA lanes sleep in their waits when the epilogue, not their
   // latency, sets the pace (prefill): then they leave the issue slots to the epilogue
   static constexpr bool PIPE_SLEEP = NG > 1;
+  // decode configurations can bin every row for the top-k (prefill ones compile no such code)
+  static constexpr bool HIST = NG == 1;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + STAGES * K_TILE_BYTES;
@@ -99,6 +101,14 @@ struct Cfg {
   static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
   static constexpr uint32_t IDESC = make_idesc(FP8 ? 0u : 1u, BM, N);
 };
+
+// Adds this warp's 32 scores (one per lane, `valid` where stored) to the row's coarse
+// histogram: lanes with equal bins are merged, one global atomic per distinct bin.
+__device__ __forceinline__ void coarse_hist_add(uint32_t* row_hist, float v, bool valid) {
+  const uint32_t bin = valid ? (order_key(__float_as_uint(v)) >> kHistShift) : 0xFFFFFFFFu;
+  const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+  if (valid && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(row_hist + bin, __popc(peers));
+}
 
 template <class C>
 __device__ __forceinline__ void issue_umma(uint32_t d_tmem, uint32_t k_stage_addr, uint32_t q_group_addr) {
@@ -398,7 +408,10 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
               relu_wsum32_reg(r0, wr_lo, a0, a1);
               relu_wsum32_reg(r1, wr_hi, a0, a1);
 #endif
-              if (key <= wi.pos0 + j) args.scores[rowoff[j] + key] = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+              const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+              const bool valid = key <= wi.pos0 + j;
+              if (valid) args.scores[rowoff[j] + key] = v;
+              if (C::HIST && args.row_hist) coarse_hist_add(args.row_hist + static_cast<int64_t>(wi.q_row0 + j) * kHistBins, v, valid);
             }
           } else if constexpr (C::H >= 32 && C::CHUNKED) {
             // many epilogue warps: one 32-column chunk in registers at a time
@@ -413,7 +426,10 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
                 tmem_ld_wait();
                 relu_wsum32(r, wq + j * C::H + c * 32, a0, a1);
               }
-              if (key <= wi.pos0 + j) args.scores[rowoff[j] + key] = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+              const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+              const bool valid = key <= wi.pos0 + j;
+              if (valid) args.scores[rowoff[j] + key] = v;
+              if (C::HIST && args.row_hist) coarse_hist_add(args.row_hist + static_cast<int64_t>(wi.q_row0 + j) * kHistBins, v, valid);
             }
           } else if constexpr (C::H >= 32) {
             // QB queries per pass: their loads are in flight behind one tcgen05.wait::ld
@@ -437,8 +453,13 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
 #pragma unroll
               for (int u = 0; u < C::QB; ++u) {
                 const int j = j0 + u * SPLIT;
-                if (live[u] && key <= wi.pos0 + j)
-                  args.scores[rowoff[j] + key] = relu_wsum<CPT>(r[u], wq + j * C::H) * kscale;
+                if (live[u]) {
+                  const float v = relu_wsum<CPT>(r[u], wq + j * C::H) * kscale;
+                  const bool valid = key <= wi.pos0 + j;
+                  if (valid) args.scores[rowoff[j] + key] = v;
+                  if (C::HIST && args.row_hist)
+                    coarse_hist_add(args.row_hist + static_cast<int64_t>(wi.q_row0 + j) * kHistBins, v, valid);
+                }
               }
             }
           } else {
@@ -453,12 +474,16 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
 #pragma unroll
               for (int u = 0; u < QPC; ++u) {
                 const int j = jc + u;
-                if (j < j_hi && key <= wi.pos0 + j) {
+                if (j < j_hi) {
                   float acc = 0.f;
 #pragma unroll
                   for (int h = 0; h < C::H; ++h)
                     acc = fmaf(wq[j * C::H + h], fmaxf(__uint_as_float(r[u * C::H + h]), 0.f), acc);
-                  args.scores[rowoff[j] + key] = acc * kscale;
+                  const float v = acc * kscale;
+                  const bool valid = key <= wi.pos0 + j;
+                  if (valid) args.scores[rowoff[j] + key] = v;
+                  if (C::HIST && args.row_hist)
+                    coarse_hist_add(args.row_hist + static_cast<int64_t>(wi.q_row0 + j) * kHistBins, v, valid);
                 }
               }
             }

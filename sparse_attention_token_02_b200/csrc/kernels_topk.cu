@@ -36,10 +36,7 @@ constexpr int kBins = kTopkBins;
 constexpr int kBinsPerThread = kBins / kThreads;
 static_assert(kBins % kThreads == 0, "bins per thread");
 
-__device__ __forceinline__ uint32_t float_to_key(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
+__device__ __forceinline__ uint32_t float_to_key(float f) { return order_key(__float_as_uint(f)); }
 
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
@@ -83,7 +80,7 @@ static_assert(kBinsPerThread == 4, "the histogram pull reads 4 bins as one uint4
 constexpr int kMaxCluster = 8;              // CTAs per row (the host never asks for more)
 
 // Keys of the threshold bin gathered into rank 0 for the rest of the selection.
-constexpr int kCandCap = 2048;
+constexpr int kCandCap = 8192;
 constexpr size_t kTopkSmemBytes = (kBins + 2 * kCandCap) * sizeof(uint32_t);
 
 // Block-wide search of a histogram held as `cnt[j]` for the bins this thread owns (bins in
@@ -153,7 +150,7 @@ topk_kernel(const TopkArgs a) {
   __syncthreads();
   grid_dependency_wait();                     // the scores come from the previous kernel
 
-  // ---- load the slice into registers as order-preserving keys (0 = absent); local key range
+  // ---- load the slice into registers as order-preserving keys (0 = absent)
   uint32_t key[EPT];
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
@@ -172,41 +169,56 @@ topk_kernel(const TopkArgs a) {
       }
     }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) {
-    atomicMin(&loc_min, kmin);
-    atomicMax(&loc_max, kmax);
-  }
-  cluster.sync();                             // #1: every CTA's key range is published
 
-  // ---- first level: bins spread over the row's key range (every CTA derives the same range)
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  {
-    uint32_t rmin[kMaxCluster], rmax[kMaxCluster];   // all remote loads in flight together
+  uint32_t bin_lo, bin_hi, n_above_total, bcount;
+  if (a.row_hist != nullptr) {
+    // ---- the logits epilogue already binned the row: the threshold bin comes straight
+    // from its coarse histogram (this CTA's 8 bins: bins 4095-8t .. 4088-8t, descending)
+    static_assert(kHistBins == 8 * kThreads, "the coarse histogram is read as 8 bins per thread");
+    const uint32_t* h = a.row_hist + static_cast<int64_t>(row) * kHistBins + (kHistBins - 8 * (tid + 1));
+    const uint4 h0 = *reinterpret_cast<const uint4*>(h);
+    const uint4 h1 = *reinterpret_cast<const uint4*>(h + 4);
+    const uint32_t c[8] = {h1.w, h1.z, h1.y, h1.x, h0.w, h0.z, h0.y, h0.x};
+    cluster.sync();                           // #1: every CTA's counters are initialised
+    find_threshold_bin<8>(c, kHistBins - 1 - 8 * tid, k, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt);
+    __syncthreads();
+    bin_lo = lvl_bin << kHistShift;
+    bin_hi = bin_lo | ((1u << kHistShift) - 1u);
+    n_above_total = lvl_above;
+    bcount = lvl_cnt;
+  } else {
+    // ---- first level from the data: bins spread over the row's key range
 #pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      rmin[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_min, r) : 0xFFFFFFFFu;
-      rmax[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_max, r) : 0u;
+    for (int o = 16; o > 0; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
     }
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      lo = min(lo, rmin[r]);
-      hi = max(hi, rmax[r]);
+    if (lane == 0) {
+      atomicMin(&loc_min, kmin);
+      atomicMax(&loc_max, kmax);
     }
-  }
-  const int bits0 = hi > lo ? 32 - __clz(hi - lo) : 0;
-  const int shift0 = bits0 > 11 ? bits0 - 11 : 0;
+    cluster.sync();                           // #1: every CTA's key range is published
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    {
+      uint32_t rmin[kMaxCluster], rmax[kMaxCluster];   // all remote loads in flight together
 #pragma unroll
-  for (int e = 0; e < EPT; ++e)
-    if (key[e]) atomicAdd(&hist[(key[e] - lo) >> shift0], 1u);
-  cluster.sync();                             // #2: every CTA's histogram is complete
-
-  // ---- every CTA sums the cluster's histograms and finds the bin of the k-th key
-  {
+      for (int r = 0; r < kMaxCluster; ++r) {
+        rmin[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_min, r) : 0xFFFFFFFFu;
+        rmax[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_max, r) : 0u;
+      }
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) {
+        lo = min(lo, rmin[r]);
+        hi = max(hi, rmax[r]);
+      }
+    }
+    const int bits0 = hi > lo ? 32 - __clz(hi - lo) : 0;
+    const int shift0 = bits0 > 11 ? bits0 - 11 : 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e)
+      if (key[e]) atomicAdd(&hist[(key[e] - lo) >> shift0], 1u);
+    cluster.sync();                           // #2: every CTA's histogram is complete
+    // every CTA sums the cluster's histograms and finds the bin of the k-th key
     uint32_t c[kBinsPerThread];
 #pragma unroll
     for (int j = 0; j < kBinsPerThread; ++j) c[j] = 0u;
@@ -226,14 +238,14 @@ topk_kernel(const TopkArgs a) {
     }
     find_threshold_bin<kBinsPerThread>(c, kBins - 1 - tid * kBinsPerThread, k, warp_sums, &lvl_bin, &lvl_above,
                                        &lvl_cnt);
+    __syncthreads();
+    bin_lo = lo + (lvl_bin << shift0);
+    const uint32_t bin_w1 = (1u << shift0) - 1u;
+    bin_hi = (hi - bin_lo) > bin_w1 ? bin_lo + bin_w1 : hi;
+    n_above_total = lvl_above;
+    bcount = lvl_cnt;
   }
-  __syncthreads();
-  const uint32_t bstar = lvl_bin, n_above_total = lvl_above, bcount = lvl_cnt;
   const uint32_t need0 = k - n_above_total;   // keys to take from the threshold bin
-  // the bin's key interval
-  const uint32_t bin_lo = lo + (bstar << shift0);
-  const uint32_t bin_w1 = (1u << shift0) - 1u;
-  const uint32_t bin_hi = (hi - bin_lo) > bin_w1 ? bin_lo + bin_w1 : hi;
 
   if (bcount <= static_cast<uint32_t>(kCandCap)) {
     // ---- fast path: write the keys above the bin, gather the bin's keys into rank 0
