@@ -69,7 +69,7 @@ struct Plan {
   std::vector<int64_t> row_off;
   std::vector<int32_t> row_pos;
   int64_t score_elems = 0;
-  int64_t hist_elems = 0;            // coarse per-row histograms (decode): T_total * kHistBins
+  bool stream_topk = false;          // decode: coarse histograms + the streaming top-k
   // top-k launches: rows grouped by (ept, cluster); short rows separately
   struct TopkClass {
     int ept, cluster;
@@ -77,13 +77,38 @@ struct Plan {
   };
   std::vector<int32_t> topk_rows;
   std::vector<TopkClass> classes;
+  std::vector<TopkChunk> chunks;     // streaming top-k (then `classes` is empty)
   int64_t short_first = 0, short_count = 0;
 };
 
 // Packs the tables into one host blob whose layout mirrors the device copy.
 struct MetaLayout {
-  size_t items = 0, cta = 0, row_off = 0, row_pos = 0, topk_rows = 0, total = 0;
+  size_t items = 0, cta = 0, row_off = 0, row_pos = 0, topk_rows = 0, chunks = 0, total = 0;
 };
+
+// Score workspace: the score rows, then (streaming top-k) the coarse histograms and row
+// counters, zeroed together every call, and the candidate buffers laid out like the rows.
+struct WsLayout {
+  size_t hist = 0, hist1 = 0, ctr = 0, zero_bytes = 0, cand_key = 0, cand_idx = 0, total = 0;
+};
+
+WsLayout ws_layout(int64_t score_elems, int64_t rows, bool stream_topk) {
+  WsLayout w;
+  size_t o = align_up(size_t(score_elems) * sizeof(float));
+  if (stream_topk) {
+    w.hist = o;
+    w.hist1 = w.hist + size_t(rows) * kHistBins * sizeof(uint32_t);
+    w.ctr = w.hist1 + size_t(rows) * kTopkBins * sizeof(uint32_t);
+    w.zero_bytes = size_t(rows) * (kHistBins + kTopkBins + 4) * sizeof(uint32_t);
+    o = align_up(o + w.zero_bytes);
+    w.cand_key = o;
+    o = align_up(o + size_t(score_elems) * sizeof(uint32_t));
+    w.cand_idx = o;
+    o = align_up(o + size_t(score_elems) * sizeof(int32_t));
+  }
+  w.total = o;
+  return w;
+}
 
 // ----------------------------------------------------------------------------- per-stream context
 
@@ -463,6 +488,25 @@ dsa_status_t plan_topk(const BatchView& v, int top_k, int sms, Plan* p) {
   return DSA_OK;
 }
 
+// Decode rows: chunks of kStreamChunk keys for the streaming top-k (no length limit).
+void plan_topk_stream(const BatchView& v, int top_k, Plan* p) {
+  p->topk_rows.clear();
+  p->classes.clear();
+  p->chunks.clear();
+  for (int64_t r = 0; r < v.total_q; ++r) {
+    const int32_t n = p->row_pos[r] + 1;
+    if (n <= top_k) {
+      p->topk_rows.push_back(static_cast<int32_t>(r));
+      continue;
+    }
+    const int32_t nch = (n + kStreamChunk - 1) / kStreamChunk;
+    for (int32_t c = 0; c < nch; ++c)
+      p->chunks.push_back(TopkChunk{static_cast<int32_t>(r), c * kStreamChunk, std::min(n, (c + 1) * kStreamChunk), nch});
+  }
+  p->short_first = 0;
+  p->short_count = static_cast<int64_t>(p->topk_rows.size());
+}
+
 MetaLayout layout_of(const Plan& p) {
   MetaLayout m;
   size_t o = 0;
@@ -471,6 +515,7 @@ MetaLayout layout_of(const Plan& p) {
   m.row_off = o;   o = align_up(o + p.row_off.size() * sizeof(int64_t));
   m.row_pos = o;   o = align_up(o + p.row_pos.size() * sizeof(int32_t));
   m.topk_rows = o; o = align_up(o + p.topk_rows.size() * sizeof(int32_t));
+  m.chunks = o;    o = align_up(o + p.chunks.size() * sizeof(TopkChunk));
   m.total = o;
   return m;
 }
@@ -483,6 +528,7 @@ std::vector<uint8_t> pack(const Plan& p, const MetaLayout& m) {
   put(m.row_off, p.row_off.data(), p.row_off.size() * sizeof(int64_t));
   put(m.row_pos, p.row_pos.data(), p.row_pos.size() * sizeof(int32_t));
   put(m.topk_rows, p.topk_rows.data(), p.topk_rows.size() * sizeof(int32_t));
+  put(m.chunks, p.chunks.data(), p.chunks.size() * sizeof(TopkChunk));
   return blob;
 }
 
@@ -558,15 +604,18 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
       plan_decode_items(v, g_sms, &np);
     else
       plan_prefill_items(v, tpa * ng, ng, g_sms, &np);
-    if (mode != Mode::Scores && (st = plan_topk(v, top_k, g_sms, &np)) != DSA_OK) return st;
-    // decode: the logits epilogue bins each row for the top-k (rows are few and long)
-    np.hist_elems = mode == Mode::Decode ? v.total_q * kHistBins : 0;
+    // decode: the logits epilogue bins each row and the top-k streams it (rows are few and long)
+    np.stream_topk = mode == Mode::Decode;
+    if (np.stream_topk)
+      plan_topk_stream(v, top_k, &np);
+    else if (mode != Mode::Scores && (st = plan_topk(v, top_k, g_sms, &np)) != DSA_OK)
+      return st;
     const MetaLayout nm = layout_of(np);
     const std::vector<uint8_t> blob = pack(np, nm);
     c->meta_valid = false;
     void* dm = nullptr;
     float* ds = nullptr;
-    const size_t ws_bytes = align_up(size_t(np.score_elems) * sizeof(float)) + size_t(np.hist_elems) * sizeof(uint32_t);
+    const size_t ws_bytes = ws_layout(np.score_elems, v.total_q, np.stream_topk).total;
     if ((st = reserve(c, nm.total, ws_bytes, &dm, &ds)) != DSA_OK) return st;
     if ((st = stage_upload(c, blob.data(), blob.size(), dm)) != DSA_OK) return st;
     c->plan = std::move(np);
@@ -581,11 +630,10 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   const MetaLayout& m = c->layout;
   float* d_scores = c->cur_scores;
   char* mb = static_cast<char*>(c->cur_meta);
-  uint32_t* d_hist = p.hist_elems
-      ? reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(d_scores) + align_up(size_t(p.score_elems) * sizeof(float)))
-      : nullptr;
-  if (d_hist)
-    DSA_CUDA_TRY(cudaMemsetAsync(d_hist, 0, size_t(p.hist_elems) * sizeof(uint32_t), stream), "cudaMemsetAsync");
+  const WsLayout wl = ws_layout(p.score_elems, v.total_q, p.stream_topk);
+  char* wsb = reinterpret_cast<char*>(d_scores);
+  uint32_t* d_hist = p.stream_topk ? reinterpret_cast<uint32_t*>(wsb + wl.hist) : nullptr;
+  if (d_hist) DSA_CUDA_TRY(cudaMemsetAsync(d_hist, 0, wl.zero_bytes, stream), "cudaMemsetAsync");
 
   CUtensorMap tk, tq;
   if ((st = encode_rows(&tk, kc->k, fp8, kc->capacity_rows, D, kKeyTile)) != DSA_OK) return st;
@@ -617,7 +665,6 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
 
   TopkArgs ta{};
   ta.scores = d_scores;
-  ta.row_hist = d_hist;
   ta.row_off = la.row_off;
   ta.row_pos = reinterpret_cast<const int32_t*>(mb + m.row_pos);
   ta.top_k = top_k;
@@ -637,6 +684,18 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     s.rows = rows + cl.first;
     s.n_rows = static_cast<int32_t>(cl.count);
     DSA_CUDA_TRY(launch_topk(s, cl.ept, cl.cluster, stream), "top-k launch");
+    ++g_launches;
+  }
+  if (!p.chunks.empty()) {
+    TopkArgs s = ta;
+    s.chunks = reinterpret_cast<const TopkChunk*>(mb + m.chunks);
+    s.n_chunks = static_cast<int32_t>(p.chunks.size());
+    s.row_hist = d_hist;
+    s.row_hist1 = reinterpret_cast<uint32_t*>(wsb + wl.hist1);
+    s.row_ctr = reinterpret_cast<uint32_t*>(wsb + wl.ctr);
+    s.cand_key = reinterpret_cast<uint32_t*>(wsb + wl.cand_key);
+    s.cand_idx = reinterpret_cast<int32_t*>(wsb + wl.cand_idx);
+    DSA_CUDA_TRY(launch_topk_stream(s, stream), "top-k (streaming) launch");
     ++g_launches;
   }
   if (g_prof[2]) DSA_CUDA_TRY(cudaEventRecordWithFlags(g_prof[2], stream, ev_flags), "cudaEventRecord");
@@ -735,9 +794,10 @@ size_t dsa_indexer_workspace_bytes(const dsa_query_t* q, const dsa_batch_t* batc
   }
   (void)top_k;
   const int64_t items = rows + tiles + 4096;   // bound on the number of work items
+  const int64_t chunks = elems / kStreamChunk + rows;   // bound on the streaming top-k's chunks
   const size_t meta = align_up(items * sizeof(LogitsItem)) + align_up((items + 2) * 4) + align_up(rows * 8) +
-                      align_up(rows * 4) + align_up(rows * 4);
-  return align_up(meta) + align_up(size_t(elems) * sizeof(float)) + size_t(rows) * kHistBins * sizeof(uint32_t);
+                      align_up(rows * 4) + align_up(rows * 4) + align_up(chunks * sizeof(TopkChunk));
+  return align_up(meta) + ws_layout(elems, rows, true).total;
 }
 
 dsa_status_t dsa_set_workspace(void* ptr, size_t bytes, void* stream_v) {

@@ -16,8 +16,9 @@ enum : int {
 };
 
 constexpr int kKeyTile = 128;       // keys per UMMA tile (the M dimension)
-// Coarse per-row score histogram built by the decode logits epilogue for the top-k:
-// bins are the top 12 bits of the order-preserving key (sign, exponent, 3 mantissa bits).
+// Coarse per-row score histogram built by the decode logits epilogue for the top-k: every
+// valid key, binned by the top 12 bits of its order-preserving key (sign, exponent and three
+// mantissa bits: eighth-octave bins).
 constexpr int kHistShift = 20;
 constexpr int kHistBins = 1 << (32 - kHistShift);
 
@@ -27,6 +28,17 @@ __host__ __device__ __forceinline__ uint32_t order_key(uint32_t float_bits) {
 }
 constexpr int kTopkThreads = 512;   // threads per top-k CTA
 constexpr int kTopkBins = 2048;     // histogram bins per refinement level
+constexpr int kStreamChunk = 4096;  // keys per CTA of the streaming (decode) top-k
+
+// One CTA of the streaming top-k: keys [begin, end) of query row `row`, which is split
+// into `n_chunks` such chunks.
+struct TopkChunk {
+  int32_t row;
+  int32_t begin;
+  int32_t end;
+  int32_t n_chunks;
+};
+static_assert(sizeof(TopkChunk) == 16, "TopkChunk layout");
 
 // One unit of logits work: `n_tok` consecutive query rows of one sequence against
 // key tiles [kt_begin, kt_end) of that sequence.
@@ -57,15 +69,22 @@ struct LogitsArgs {
 
 struct TopkArgs {
   const float* scores;
-  const uint32_t* row_hist;  // coarse histograms from the logits epilogue, or nullptr
   const int64_t* row_off;
   const int32_t* row_pos;    // [T_total]: position p of each query row (valid keys 0..p)
-  const int32_t* rows;       // rows handled by this launch
+  const int32_t* rows;       // rows handled by this launch (cluster and short kernels)
   int32_t n_rows;
   int32_t top_k;
   int32_t* out_idx;
   float* out_score;
   int* err;
+  // streaming kernel only
+  const TopkChunk* chunks;   // [n_chunks], the chunks of a row consecutive
+  int32_t n_chunks;
+  const uint32_t* row_hist;  // [T_total, kHistBins] coarse histograms from the logits epilogue
+  uint32_t* row_hist1;       // [T_total, kTopkBins] zeroed: level-1 histograms of each row's threshold bin
+  uint32_t* row_ctr;         // [T_total, 4] zeroed: bin keys gathered, keys written above the bin, chunks done
+  uint32_t* cand_key;        // gathered bin keys of row r at cand_key + row_off[r]
+  int32_t* cand_idx;         // their positions, same layout
 };
 
 // ----------------------------------------------------------------------------- launchers
@@ -87,6 +106,9 @@ bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng);
 // Top-k over rows longer than top_k: one cluster of `cluster` CTAs per row,
 // `ept` keys per thread held in registers.
 cudaError_t launch_topk(const TopkArgs& a, int ept, int cluster, cudaStream_t stream);
+// Rows whose coarse histogram the logits epilogue built: one CTA per chunk of kStreamChunk
+// keys, the last CTA of a row finishing the selection inside the threshold bin.
+cudaError_t launch_topk_stream(const TopkArgs& a, cudaStream_t stream);
 // Rows with at most top_k candidates: every causal position, then padding.
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream);
 

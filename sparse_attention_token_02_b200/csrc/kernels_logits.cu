@@ -102,12 +102,14 @@ struct Cfg {
   static constexpr uint32_t IDESC = make_idesc(FP8 ? 0u : 1u, BM, N);
 };
 
-// Adds this warp's 32 scores (one per lane, `valid` where stored) to the row's coarse
-// histogram: lanes with equal bins are merged, one global atomic per distinct bin.
+// Counts this warp's 32 scores (one per lane, invalid lanes skipped) in the row's coarse
+// histogram.  Lanes whose keys share a bin are merged first (one atomic per distinct bin
+// per warp): a row's scores crowd into a few bins, and same-address atomics serialise at
+// the L2.  Called by all 32 lanes together.
 __device__ __forceinline__ void coarse_hist_add(uint32_t* row_hist, float v, bool valid) {
-  const uint32_t bin = valid ? (order_key(__float_as_uint(v)) >> kHistShift) : 0xFFFFFFFFu;
+  const uint32_t bin = valid ? order_key(__float_as_uint(v)) >> kHistShift : 0xFFFFFFFFu;
   const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-  if (valid && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(row_hist + bin, __popc(peers));
+  if (valid && static_cast<int>(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(row_hist + bin, __popc(peers));
 }
 
 template <class C>
@@ -123,6 +125,29 @@ __device__ __forceinline__ void issue_umma(uint32_t d_tmem, uint32_t k_stage_add
         umma_f8(d_tmem, a, b, C::IDESC, acc);
       else
         umma_f16(d_tmem, a, b, C::IDESC, acc);
+    }
+  }
+}
+
+// Two independent tiles (separate accumulators) issued with their K steps interleaved,
+// so no UMMA waits for the one just before it to finish its read-modify-write of D.
+template <class C>
+__device__ __forceinline__ void issue_umma_pair(uint32_t d0, uint32_t k0, uint32_t d1, uint32_t k1, uint32_t q) {
+#pragma unroll
+  for (int kb = 0; kb < C::KB; ++kb) {
+#pragma unroll
+    for (int ks = 0; ks < C::KSTEPS; ++ks) {
+      const uint64_t b = sdesc_kmajor_sw128(q + kb * C::Q_BLOCK_BYTES + ks * 32);
+      const uint64_t a0 = sdesc_kmajor_sw128(k0 + kb * C::K_BLOCK_BYTES + ks * 32);
+      const uint64_t a1 = sdesc_kmajor_sw128(k1 + kb * C::K_BLOCK_BYTES + ks * 32);
+      const uint32_t acc = (kb | ks) != 0;
+      if constexpr (C::FP8) {
+        umma_f8(d0, a0, b, C::IDESC, acc);
+        umma_f8(d1, a1, b, C::IDESC, acc);
+      } else {
+        umma_f16(d0, a0, b, C::IDESC, acc);
+        umma_f16(d1, a1, b, C::IDESC, acc);
+      }
     }
   }
 }
@@ -285,6 +310,38 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
         const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
         if (!DSA_TIMED(7, mbar_wait<C::PIPE_SLEEP>(q_full, item_iter & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
+        if constexpr (C::NG == 1) {
+          // one accumulator per tile: issue tiles in pairs, their UMMA chains interleaved
+          static_assert(C::NBUF >= 2 && C::STAGES >= 2, "a pair needs two accumulators and two stages");
+          for (int kt = wi.kt_begin; kt < wi.kt_end && ok;) {
+            const bool two = kt + 1 < wi.kt_end;
+            const int s0 = k_iter % C::STAGES, s1 = (k_iter + 1) % C::STAGES;
+            const int b0 = acc_iter % C::NBUF, b1 = (acc_iter + 1) % C::NBUF;
+            if (!DSA_TIMED(1, mbar_wait(&k_full[s0], (k_iter / C::STAGES) & 1, abort_flag)) ||
+                (two && !DSA_TIMED(1, mbar_wait(&k_full[s1], ((k_iter + 1) / C::STAGES) & 1, abort_flag))) ||
+                !DSA_TIMED(2, mbar_wait(&acc_empty[b0], ((acc_iter / C::NBUF) & 1) ^ 1, abort_flag)) ||
+                (two && !DSA_TIMED(2, mbar_wait(&acc_empty[b1], (((acc_iter + 1) / C::NBUF) & 1) ^ 1, abort_flag)))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kaddr0 = smem_base + C::OFF_K + s0 * C::K_TILE_BYTES;
+            const uint32_t kaddr1 = smem_base + C::OFF_K + s1 * C::K_TILE_BYTES;
+            if (two)
+              issue_umma_pair<C>(tmem_base + b0 * C::ACC_COLS, kaddr0, tmem_base + b1 * C::ACC_COLS, kaddr1,
+                                 smem_base + C::OFF_Q);
+            else
+              issue_umma<C>(tmem_base + b0 * C::ACC_COLS, kaddr0, smem_base + C::OFF_Q);
+            umma_commit(&acc_full[b0]);
+            if (two) umma_commit(&acc_full[b1]);
+            umma_commit(&k_empty[s0]);
+            if (two) umma_commit(&k_empty[s1]);
+            const int adv = two ? 2 : 1;
+            kt += adv;
+            k_iter += adv;
+            acc_iter += adv;
+          }
+        } else
         for (int kt = wi.kt_begin; kt < wi.kt_end && ok; ++kt, ++k_iter) {
           const int s = k_iter % C::STAGES;
           if (!DSA_TIMED(1, mbar_wait<C::PIPE_SLEEP>(&k_full[s], (k_iter / C::STAGES) & 1, abort_flag))) { ok = false; break; }

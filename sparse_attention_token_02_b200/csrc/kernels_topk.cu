@@ -46,6 +46,7 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 // Exclusive prefix sum over the CTA's threads (in threadIdx order); also returns the total.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n_warps = blockDim.x >> 5;
   uint32_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -55,20 +56,22 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    uint32_t s = lane < kWarps ? warp_sums[lane] : 0u;
+    uint32_t s = lane < n_warps ? warp_sums[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    if (lane < kWarps) warp_sums[lane] = s;   // inclusive warp prefix
+    if (lane < n_warps) warp_sums[lane] = s;   // inclusive warp prefix
   }
   __syncthreads();
-  total = warp_sums[kWarps - 1];
+  total = warp_sums[n_warps - 1];
   const uint32_t before = warp == 0 ? 0u : warp_sums[warp - 1];
   __syncthreads();                            // warp_sums may be reused right after
   return before + x - v;
 }
+
+constexpr uint32_t kNotFound = 0xFFFFFFFFu;
 
 struct SelectState {
   uint32_t lo, hi;      // candidate key interval
@@ -106,6 +109,101 @@ __device__ __forceinline__ void find_threshold_bin(const uint32_t (&cnt)[PER], u
   }
 }
 
+// Calls f(key, index) for candidates [0, m), each thread taking every NT-th one.  Reads
+// go in batches of CPT per thread, all loads of a batch issued before any is used: global
+// candidates cost an L2 round trip each, which a one-at-a-time loop would serialise.
+template <bool kGlobal, bool kWithIdx, int NT, int CPT, class F>
+__device__ __forceinline__ void for_candidates(const uint32_t* ck, const int32_t* ci, uint32_t m, F&& f) {
+  for (uint32_t b0 = 0; b0 < m; b0 += NT * CPT) {
+    uint32_t kk[CPT];
+    int32_t ix[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const uint32_t i = b0 + j * NT + threadIdx.x;
+      kk[j] = 0u;
+      ix[j] = 0;
+      if (i < m) {
+        kk[j] = kGlobal ? __ldcg(ck + i) : ck[i];
+        if (kWithIdx) ix[j] = kGlobal ? __ldcg(ci + i) : ci[i];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < CPT; ++j)
+      if (b0 + j * NT + threadIdx.x < m) f(kk[j], ix[j]);
+  }
+}
+
+// One CTA, all its threads: among the m gathered keys in [lo, hi] (candidates in this
+// CTA's shared memory, or with kGlobalCand in global memory, read through the L2 since
+// other CTAs wrote them), write the `need` largest to slots [base, base + need) of the row.
+// Exact: CTA-local histogram levels narrow [lo, hi] by >= 2^10 per level; keys above the
+// final interval are taken, then `need` of its keys (a single tied value if not resolved).
+// Returns false if the counts turn out inconsistent (nothing is written past the row).
+template <bool kGlobalCand, int NT>
+__device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, uint32_t m, uint32_t lo,
+                             uint32_t hi, uint32_t need, uint32_t base, int32_t* oi, float* os, uint32_t* hist,
+                             uint32_t* warp_sums, uint32_t* lvl_bin, uint32_t* lvl_above, uint32_t* lvl_cnt,
+                             uint32_t* ctr_a, uint32_t* ctr_b) {
+  constexpr int PER = kBins / NT;
+  constexpr int CPT = kGlobalCand ? 8 : 1;
+  const int tid = threadIdx.x;
+  SelectState ls;
+  ls.lo = lo;
+  ls.hi = hi;
+  ls.need = need;
+  ls.done = need == m ? 1u : 0u;
+  for (int level = 0; level < 4 && !ls.done; ++level) {
+    if (ls.lo == ls.hi) { ls.done = 2; break; }
+    const int bits = 32 - __clz(ls.hi - ls.lo);
+    const int shift = bits > 11 ? bits - 11 : 0;
+    for (int b = tid; b < kBins; b += NT) hist[b] = 0u;
+    __syncthreads();
+    for_candidates<kGlobalCand, false, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t) {
+      if (kk >= ls.lo && kk <= ls.hi) atomicAdd(&hist[(kk - ls.lo) >> shift], 1u);
+    });
+    __syncthreads();
+    uint32_t c[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) c[j] = hist[kBins - 1 - (tid * PER + j)];
+    if (tid == 0) *lvl_bin = kNotFound;
+    find_threshold_bin<PER>(c, kBins - 1 - tid * PER, ls.need, warp_sums, lvl_bin, lvl_above, lvl_cnt);
+    __syncthreads();
+    if (*lvl_bin == kNotFound) return false;
+    SelectState ns;
+    ns.lo = ls.lo + (*lvl_bin << shift);
+    const uint32_t width_m1 = (1u << shift) - 1u;
+    ns.hi = (ls.hi - ns.lo) > width_m1 ? ns.lo + width_m1 : ls.hi;
+    ns.need = ls.need - *lvl_above;
+    ns.done = *lvl_cnt == ns.need ? 1u : 0u;
+    ls = ns;
+    __syncthreads();
+  }
+  if (!ls.done) ls.done = 2;                  // unreachable: >= 10 bits resolved per level
+  if (tid == 0) {
+    *ctr_a = 0u;
+    *ctr_b = 0u;
+  }
+  __syncthreads();
+  const uint32_t first_in = base + (need - ls.need);     // slots of interval keys start here
+  for_candidates<kGlobalCand, true, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t ix) {
+    if (kk > ls.hi) {
+      const uint32_t slot = base + atomicAdd(ctr_a, 1u);
+      if (slot < first_in) {
+        oi[slot] = ix;
+        os[slot] = key_to_float(kk);
+      }
+    } else if (kk >= ls.lo) {
+      const uint32_t t = atomicAdd(ctr_b, 1u);
+      if (t < ls.need) {
+        oi[first_in + t] = ix;
+        os[first_in + t] = key_to_float(kk);
+      }
+    }
+  });
+  __syncthreads();
+  return *ctr_a == need - ls.need && *ctr_b >= ls.need && !(ls.done == 1 && *ctr_b != ls.need);
+}
+
 template <int EPT>
 __global__ void __launch_bounds__(kThreads, EPT <= 8 ? 2 : 1)
 topk_kernel(const TopkArgs a) {
@@ -139,6 +237,8 @@ topk_kernel(const TopkArgs a) {
 
   uint32_t* cnt_above0 = cluster.map_shared_rank(&cnt_above, 0);
   uint32_t* cnt_cand0 = cluster.map_shared_rank(&cnt_cand, 0);
+  uint32_t* ck0 = cluster.map_shared_rank(cand_key, 0);
+  int32_t* ci0 = cluster.map_shared_rank(cand_idx, 0);
 
   for (int b = tid; b < kBins; b += kThreads) hist[b] = 0u;
   if (tid == 0) {
@@ -146,6 +246,9 @@ topk_kernel(const TopkArgs a) {
     cnt_cand = 0u;
     loc_min = 0xFFFFFFFFu;
     loc_max = 0u;
+    lvl_bin = kNotFound;                      // stays so if a histogram cannot reach its target
+    lvl_above = 0u;
+    lvl_cnt = 0u;
   }
   __syncthreads();
   grid_dependency_wait();                     // the scores come from the previous kernel
@@ -170,54 +273,38 @@ topk_kernel(const TopkArgs a) {
     }
   }
 
-  uint32_t bin_lo, bin_hi, n_above_total, bcount;
-  if (a.row_hist != nullptr) {
-    // ---- the logits epilogue already binned the row: the threshold bin comes straight
-    // from its coarse histogram (this CTA's 8 bins: bins 4095-8t .. 4088-8t, descending)
-    static_assert(kHistBins == 8 * kThreads, "the coarse histogram is read as 8 bins per thread");
-    const uint32_t* h = a.row_hist + static_cast<int64_t>(row) * kHistBins + (kHistBins - 8 * (tid + 1));
-    const uint4 h0 = *reinterpret_cast<const uint4*>(h);
-    const uint4 h1 = *reinterpret_cast<const uint4*>(h + 4);
-    const uint32_t c[8] = {h1.w, h1.z, h1.y, h1.x, h0.w, h0.z, h0.y, h0.x};
-    cluster.sync();                           // #1: every CTA's counters are initialised
-    find_threshold_bin<8>(c, kHistBins - 1 - 8 * tid, k, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt);
-    __syncthreads();
-    bin_lo = lvl_bin << kHistShift;
-    bin_hi = bin_lo | ((1u << kHistShift) - 1u);
-    n_above_total = lvl_above;
-    bcount = lvl_cnt;
-  } else {
-    // ---- first level from the data: bins spread over the row's key range
+  // ---- data-driven first level: bins spread over the row's key range
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    atomicMin(&loc_min, kmin);
+    atomicMax(&loc_max, kmax);
+  }
+  cluster.sync();                             // every CTA's key range is published
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  {
+    uint32_t rmin[kMaxCluster], rmax[kMaxCluster];   // all remote loads in flight together
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      rmin[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_min, r) : 0xFFFFFFFFu;
+      rmax[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_max, r) : 0u;
     }
-    if (lane == 0) {
-      atomicMin(&loc_min, kmin);
-      atomicMax(&loc_max, kmax);
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      lo = min(lo, rmin[r]);
+      hi = max(hi, rmax[r]);
     }
-    cluster.sync();                           // #1: every CTA's key range is published
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    {
-      uint32_t rmin[kMaxCluster], rmax[kMaxCluster];   // all remote loads in flight together
+  }
+  const int bits0 = hi > lo ? 32 - __clz(hi - lo) : 0;
+  const int shift0 = bits0 > 11 ? bits0 - 11 : 0;
 #pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) {
-        rmin[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_min, r) : 0xFFFFFFFFu;
-        rmax[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_max, r) : 0u;
-      }
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) {
-        lo = min(lo, rmin[r]);
-        hi = max(hi, rmax[r]);
-      }
-    }
-    const int bits0 = hi > lo ? 32 - __clz(hi - lo) : 0;
-    const int shift0 = bits0 > 11 ? bits0 - 11 : 0;
-#pragma unroll
-    for (int e = 0; e < EPT; ++e)
-      if (key[e]) atomicAdd(&hist[(key[e] - lo) >> shift0], 1u);
-    cluster.sync();                           // #2: every CTA's histogram is complete
+  for (int e = 0; e < EPT; ++e)
+    if (key[e]) atomicAdd(&hist[(key[e] - lo) >> shift0], 1u);
+  cluster.sync();                             // every CTA's histogram is complete
+  {
     // every CTA sums the cluster's histograms and finds the bin of the k-th key
     uint32_t c[kBinsPerThread];
 #pragma unroll
@@ -238,17 +325,23 @@ topk_kernel(const TopkArgs a) {
     }
     find_threshold_bin<kBinsPerThread>(c, kBins - 1 - tid * kBinsPerThread, k, warp_sums, &lvl_bin, &lvl_above,
                                        &lvl_cnt);
-    __syncthreads();
-    bin_lo = lo + (lvl_bin << shift0);
-    const uint32_t bin_w1 = (1u << shift0) - 1u;
-    bin_hi = (hi - bin_lo) > bin_w1 ? bin_lo + bin_w1 : hi;
-    n_above_total = lvl_above;
-    bcount = lvl_cnt;
   }
+  __syncthreads();
+  if (lvl_bin == kNotFound) {
+    // The histogram holds fewer than top_k keys, which the row's data cannot produce:
+    // record the fault and write nothing (every CTA of the cluster takes this branch).
+    cluster.sync();                           // no CTA still reads another's shared memory
+    if (crank == 0 && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    return;
+  }
+  const uint32_t bin_lo = lo + (lvl_bin << shift0);
+  const uint32_t bin_w1 = (1u << shift0) - 1u;
+  const uint32_t bin_hi = (hi - bin_lo) > bin_w1 ? bin_lo + bin_w1 : hi;
+  const uint32_t n_above_total = lvl_above, bcount = lvl_cnt;
   const uint32_t need0 = k - n_above_total;   // keys to take from the threshold bin
 
   if (bcount <= static_cast<uint32_t>(kCandCap)) {
-    // ---- fast path: write the keys above the bin, gather the bin's keys into rank 0
+    // ---- write the keys above the bin, gather the bin's keys into rank 0
     uint32_t n_up = 0, n_in = 0;
 #pragma unroll
     for (int e = 0; e < EPT; ++e) {
@@ -263,8 +356,6 @@ topk_kernel(const TopkArgs a) {
       base_cand = tot_in ? atomicAdd(cnt_cand0, tot_in) : 0u;
     }
     __syncthreads();
-    uint32_t* ck0 = cluster.map_shared_rank(cand_key, 0);
-    int32_t* ci0 = cluster.map_shared_rank(cand_idx, 0);
     uint32_t iu = base_above + pre_up, ic = base_cand + pre_in;
 #pragma unroll
     for (int v = 0; v < EPT / 4; ++v) {
@@ -289,70 +380,10 @@ topk_kernel(const TopkArgs a) {
     }
     cluster.sync();                           // rank 0 holds the whole bin; counters are final
     if (crank != 0) return;                   // nobody reads another CTA's memory after this point
-
-    // ---- rank 0 alone: pick need0 of the bcount gathered keys (exact, CTA-local levels)
-    const uint32_t m = bcount;
-    SelectState ls;
-    ls.lo = bin_lo;
-    ls.hi = bin_hi;
-    ls.need = need0;
-    ls.done = need0 == m ? 1u : 0u;
-    for (int level = 0; level < 4 && !ls.done; ++level) {
-      if (ls.lo == ls.hi) { ls.done = 2; break; }
-      const int bits = 32 - __clz(ls.hi - ls.lo);
-      const int shift = bits > 11 ? bits - 11 : 0;
-      for (int b = tid; b < kBins; b += kThreads) hist[b] = 0u;
-      __syncthreads();
-      for (uint32_t i = tid; i < m; i += kThreads) {
-        const uint32_t kk = cand_key[i];
-        if (kk >= ls.lo && kk <= ls.hi) atomicAdd(&hist[(kk - ls.lo) >> shift], 1u);
-      }
-      __syncthreads();
-      uint32_t c[kBinsPerThread];
-#pragma unroll
-      for (int j = 0; j < kBinsPerThread; ++j) c[j] = hist[kBins - 1 - (tid * kBinsPerThread + j)];
-      find_threshold_bin<kBinsPerThread>(c, kBins - 1 - tid * kBinsPerThread, ls.need, warp_sums, &lvl_bin,
-                                         &lvl_above, &lvl_cnt);
-      __syncthreads();
-      const uint32_t b2 = lvl_bin;
-      SelectState ns;
-      ns.lo = ls.lo + (b2 << shift);
-      const uint32_t width_m1 = (1u << shift) - 1u;
-      ns.hi = (ls.hi - ns.lo) > width_m1 ? ns.lo + width_m1 : ls.hi;
-      ns.need = ls.need - lvl_above;
-      ns.done = lvl_cnt == ns.need ? 1u : 0u;
-      ls = ns;
-      __syncthreads();
-    }
-    if (!ls.done) ls.done = 2;                // unreachable: >= 10 bits resolved per level
-    // candidates above the final interval, then ls.need keys of the interval (ties: any)
-    if (tid == 0) {
-      cnt_above = 0u;                         // reused as slot counters for this CTA only
-      cnt_cand = 0u;
-    }
-    __syncthreads();
-    const uint32_t first_in = n_above_total + (need0 - ls.need);   // slots of interval keys start here
-    for (uint32_t i = tid; i < m; i += kThreads) {
-      const uint32_t kk = cand_key[i];
-      if (kk > ls.hi) {
-        const uint32_t slot = n_above_total + atomicAdd(&cnt_above, 1u);
-        if (slot < first_in) {
-          oi[slot] = cand_idx[i];
-          os[slot] = key_to_float(kk);
-        }
-      } else if (kk >= ls.lo) {
-        const uint32_t t = atomicAdd(&cnt_cand, 1u);
-        if (t < ls.need) {
-          oi[first_in + t] = cand_idx[i];
-          os[first_in + t] = key_to_float(kk);
-        }
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      const bool bad = cnt_above != need0 - ls.need || cnt_cand < ls.need || (ls.done == 1 && cnt_cand != ls.need);
-      if (bad) record_error(a.err, DSA_DEVERR_TOPK, row);
-    }
+    const bool above_ok = cnt_above == n_above_total && cnt_cand == bcount;
+    const bool ok = rank0_select<false, kThreads>(cand_key, cand_idx, bcount, bin_lo, bin_hi, need0, n_above_total, oi, os, hist,
+                                 warp_sums, &lvl_bin, &lvl_above, &lvl_cnt, &base_above, &base_cand);
+    if ((!ok || !above_ok) && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
     return;
   }
 
@@ -388,10 +419,15 @@ topk_kernel(const TopkArgs a) {
       uint32_t c[kBinsPerThread];
 #pragma unroll
       for (int j = 0; j < kBinsPerThread; ++j) c[j] = hist[kBins - 1 - (tid * kBinsPerThread + j)];
+      if (tid == 0) lvl_bin = kNotFound;
       find_threshold_bin<kBinsPerThread>(c, kBins - 1 - tid * kBinsPerThread, s.need, warp_sums, &lvl_bin,
                                          &lvl_above, &lvl_cnt);
       __syncthreads();
-      if (tid == 0) {
+      if (tid == 0 && lvl_bin == kNotFound) {
+        SelectState bad = s;
+        bad.done = 3;                         // inconsistent counts: every CTA stops below
+        st = bad;
+      } else if (tid == 0) {
         SelectState ns;
         ns.lo = s.lo + (lvl_bin << shift);
         const uint32_t width_m1 = (1u << shift) - 1u;
@@ -406,6 +442,11 @@ topk_kernel(const TopkArgs a) {
     if (s.done) break;
   }
   if (!s.done) s.done = 2;
+  if (s.done == 3) {
+    cluster.sync();                           // no CTA still reads rank 0's state
+    if (crank == 0 && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    return;
+  }
 
   uint32_t n_up = 0, n_in = 0;
 #pragma unroll
@@ -449,6 +490,199 @@ topk_kernel(const TopkArgs a) {
     const bool bad = cnt_above != n_sel_above || cnt_cand < s.need || (s.done == 1 && cnt_cand != s.need);
     if (bad) record_error(a.err, DSA_DEVERR_TOPK, row);
   }
+}
+
+// ---- streaming top-k for rows whose coarse histogram the logits epilogue built.
+// The histogram fixes, before any score is read, the bin B that holds the k-th largest
+// key and the number of keys above B, so a row's keys need not meet in one place: every
+// CTA streams one chunk of kStreamChunk scores, writes the keys above B straight to the
+// row's output (slots from a per-row counter), appends the keys inside B to the row's
+// candidate buffer and counts them in a per-row level-1 histogram of B (2048 sub-bins).
+// Only the candidates and their counts must be visible before a chunk takes its ticket; the
+// keys above B are written after it.  The CTA that finishes a row's last chunk reads that
+// histogram, finds the sub-bin S of the remaining keys, takes the candidates above S in one
+// pass and selects inside S in shared memory.  No CTA waits for another.
+constexpr int kStreamThreads = 256;
+constexpr int kStreamEPT = kStreamChunk / kStreamThreads;
+constexpr int kStreamPer0 = kHistBins / kStreamThreads;  // coarse histogram bins per thread
+constexpr int kStreamPer1 = kBins / kStreamThreads;      // level-1 histogram bins per thread
+constexpr int kSubShift = kHistShift - 11;               // level-1 sub-bin width 2^kSubShift
+constexpr int kSubCap = 1024;                            // sub-bin keys held in shared memory
+static_assert(kStreamEPT % 4 == 0 && kStreamPer0 % 4 == 0 && kStreamPer1 % 4 == 0, "chunk and histogram split");
+static_assert((1u << (kHistShift - kSubShift)) == static_cast<uint32_t>(kBins), "one level-1 bin per sub-bin");
+
+// PER consecutive bins starting at h, returned in descending bin order.
+template <int PER>
+__device__ __forceinline__ void load_bins_desc(const uint32_t* h, uint32_t (&c)[PER]) {
+#pragma unroll
+  for (int q = 0; q < PER / 4; ++q) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(h + 4 * q));
+    c[PER - 1 - 4 * q] = v.x;
+    c[PER - 2 - 4 * q] = v.y;
+    c[PER - 3 - 4 * q] = v.z;
+    c[PER - 4 - 4 * q] = v.w;
+  }
+}
+
+__global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkArgs a) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t sub_key[kSubCap];
+  __shared__ int32_t sub_idx[kSubCap];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t lvl_bin, lvl_above, lvl_cnt, ctr_a, ctr_b;
+  __shared__ unsigned long long bases;
+  __shared__ int is_last;
+  const int tid = threadIdx.x;
+  const TopkChunk ch = a.chunks[blockIdx.x];
+  const int row = ch.row;
+  const int n = a.row_pos[row] + 1;
+  const int64_t off = a.row_off[row];
+  const float* src = a.scores + off;
+  const uint32_t k = static_cast<uint32_t>(a.top_k);
+  int32_t* oi = a.out_idx + static_cast<int64_t>(row) * a.top_k;
+  float* os = a.out_score + static_cast<int64_t>(row) * a.top_k;
+  // row counters: [0] bin keys gathered, [1] keys written above the bin (one 64-bit word), [2] chunks done
+  uint32_t* ctr = a.row_ctr + 4 * static_cast<int64_t>(row);
+  uint32_t* sub_hist = a.row_hist1 + static_cast<int64_t>(row) * kBins;
+  if (tid == 0) lvl_bin = kNotFound;          // published by the scan's barriers below
+  grid_dependency_wait();                     // scores and histograms come from the previous kernel
+
+  uint32_t c0[kStreamPer0];
+  load_bins_desc<kStreamPer0>(a.row_hist + static_cast<int64_t>(row) * kHistBins + (kHistBins - kStreamPer0 * (tid + 1)),
+                              c0);
+  uint32_t key[kStreamEPT];
+#pragma unroll
+  for (int v = 0; v < kStreamEPT / 4; ++v) {
+    const int i = ch.begin + (v * kStreamThreads + tid) * 4;
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < ch.end) f = __ldcs(reinterpret_cast<const float4*>(src + i));
+    const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) key[v * 4 + e] = (i + e < ch.end) ? float_to_key(fv[e]) : 0u;
+  }
+  find_threshold_bin<kStreamPer0>(c0, kHistBins - 1 - kStreamPer0 * tid, k, warp_sums, &lvl_bin, &lvl_above,
+                                  &lvl_cnt);
+  __syncthreads();
+  if (lvl_bin == kNotFound) {
+    // fewer than top_k keys counted for a row longer than top_k: every CTA of the row
+    // lands here, so no CTA of it takes the ticket and nothing is written
+    if (tid == 0 && ch.begin == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    return;
+  }
+  const uint32_t bin_lo = lvl_bin << kHistShift;
+  const uint32_t bin_hi = bin_lo | ((1u << kHistShift) - 1u);
+  const uint32_t n_above_total = lvl_above, bcount = lvl_cnt;
+  const uint32_t cap = min(bcount, static_cast<uint32_t>(n));   // the row's candidate room is >= n
+
+  // one scan of both counts (each < 2^16 per CTA) and one 64-bit atomic for both bases
+  uint32_t n_up = 0, n_in = 0;
+#pragma unroll
+  for (int e = 0; e < kStreamEPT; ++e) {
+    n_up += key[e] > bin_hi;
+    n_in += key[e] >= bin_lo && key[e] <= bin_hi;
+  }
+  uint32_t tot;
+  const uint32_t pre = block_exclusive_scan((n_up << 16) | n_in, warp_sums, tot);
+  if (tid == 0)
+    bases = tot ? atomicAdd(reinterpret_cast<unsigned long long*>(ctr),
+                            (static_cast<unsigned long long>(tot >> 16) << 32) | (tot & 0xFFFFu))
+                : 0ull;
+  __syncthreads();
+  uint32_t ic = static_cast<uint32_t>(bases) + (pre & 0xFFFFu);
+#pragma unroll
+  for (int v = 0; v < kStreamEPT / 4; ++v) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t kk = key[v * 4 + e];
+      if (kk >= bin_lo && kk <= bin_hi) {
+        if (ic < cap) {
+          a.cand_key[off + ic] = kk;
+          a.cand_idx[off + ic] = ch.begin + (v * kStreamThreads + tid) * 4 + e;
+        }
+        ++ic;
+        atomicAdd(sub_hist + ((kk - bin_lo) >> kSubShift), 1u);
+      }
+    }
+  }
+  __threadfence();                            // this chunk's candidates before its ticket
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(ctr + 2, 1u) == static_cast<uint32_t>(ch.n_chunks - 1);
+  // the keys above the bin: nobody reads them in this kernel
+  uint32_t iu = static_cast<uint32_t>(bases >> 32) + (pre >> 16);
+#pragma unroll
+  for (int v = 0; v < kStreamEPT / 4; ++v) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t kk = key[v * 4 + e];
+      if (kk > bin_hi) {
+        if (iu < n_above_total) {
+          oi[iu] = ch.begin + (v * kStreamThreads + tid) * 4 + e;
+          os[iu] = key_to_float(kk);
+        }
+        ++iu;
+      }
+    }
+  }
+  __syncthreads();
+  if (!is_last) return;
+
+  // ---- the row's last chunk: every other chunk's writes are visible after this fence
+  __threadfence();
+  const unsigned long long got = __ldcg(reinterpret_cast<const unsigned long long*>(ctr));
+  if (static_cast<uint32_t>(got >> 32) != n_above_total || static_cast<uint32_t>(got) != bcount) {
+    if (tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    return;
+  }
+  const uint32_t need0 = k - n_above_total;
+  if (tid == 0) lvl_bin = kNotFound;
+  uint32_t c1[kStreamPer1];
+  load_bins_desc<kStreamPer1>(sub_hist + (kBins - kStreamPer1 * (tid + 1)), c1);
+  find_threshold_bin<kStreamPer1>(c1, kBins - 1 - kStreamPer1 * tid, need0, warp_sums, &lvl_bin, &lvl_above,
+                                  &lvl_cnt);
+  __syncthreads();
+  if (lvl_bin == kNotFound) {
+    if (tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    return;
+  }
+  const uint32_t above1 = lvl_above, cnt1 = lvl_cnt;
+  const uint32_t sub_lo = bin_lo + (lvl_bin << kSubShift);
+  const uint32_t sub_hi = sub_lo + ((1u << kSubShift) - 1u);
+  bool ok;
+  if (cnt1 <= static_cast<uint32_t>(kSubCap)) {
+    if (tid == 0) {
+      ctr_a = 0u;
+      ctr_b = 0u;
+    }
+    __syncthreads();
+    for_candidates<true, true, kStreamThreads, 8>(a.cand_key + off, a.cand_idx + off, bcount,
+                                                   [&](uint32_t kk, int32_t ix) {
+      if (kk > sub_hi) {
+        const uint32_t t = atomicAdd(&ctr_a, 1u);
+        if (t < above1) {
+          oi[n_above_total + t] = ix;
+          os[n_above_total + t] = key_to_float(kk);
+        }
+      } else if (kk >= sub_lo) {
+        const uint32_t t = atomicAdd(&ctr_b, 1u);
+        if (t < static_cast<uint32_t>(kSubCap)) {
+          sub_key[t] = kk;
+          sub_idx[t] = ix;
+        }
+      }
+    });
+    __syncthreads();
+    const bool pass_ok = ctr_a == above1 && ctr_b == cnt1;
+    __syncthreads();                          // every thread has read the counters
+    ok = pass_ok && rank0_select<false, kStreamThreads>(sub_key, sub_idx, cnt1, sub_lo, sub_hi, need0 - above1,
+                                                         n_above_total + above1, oi, os, hist, warp_sums, &lvl_bin,
+                                                         &lvl_above, &lvl_cnt, &ctr_a, &ctr_b);
+  } else {
+    // a crowded sub-bin (many equal scores): refine over all the row's candidates
+    ok = rank0_select<true, kStreamThreads>(a.cand_key + off, a.cand_idx + off, bcount, bin_lo, bin_hi, need0,
+                                            n_above_total, oi, os, hist, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt,
+                                            &ctr_a, &ctr_b);
+  }
+  if (!ok && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
 }
 
 // Rows whose whole causal history fits in top_k: every position, then -1 / -inf.
@@ -510,6 +744,20 @@ cudaError_t launch_topk(const TopkArgs& a, int ept, int cluster, cudaStream_t st
     case 32: return launch_ept<32>(a, cluster, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_topk_stream(const TopkArgs& a, cudaStream_t stream) {
+  if (a.n_chunks <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.n_chunks), 1, 1);
+  cfg.blockDim = dim3(kStreamThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_stream_kernel, a);
 }
 
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream) {

@@ -235,6 +235,32 @@ def test_edge_ties_and_zero_and_negative_weights():
         _check(up, idx, sc, [0, 1, 99, 100, 101, 500, 1499])
 
 
+def test_edge_decode_ties_zero_and_negative_weights():
+    # decode rows over several chunks of the streaming top-k; with zero weights every
+    # score is 0, so the threshold bin holds the whole row and the choice is all ties
+    lens = (9000, 4100, 2049, 8193)
+    wl = W.scaled(W.decode(), seq_lens=lens, q_lens=(2,) * len(lens), top_k=300, seed=41)
+    inp = W.make_inputs(wl)
+    rng = np.random.default_rng(2)
+    inp["k_bits"] = [W.f32_to_bf16_bits(rng.integers(-2, 3, (L, 128)).astype(np.float32)) for L in lens]
+    inp["q_bits"] = W.f32_to_bf16_bits(rng.integers(-1, 2, (wl.total_q, 64, 128)).astype(np.float32))
+    T = wl.total_q
+    for w in (np.full((T, 64), 1.0 / 64, np.float32), np.zeros((T, 64), np.float32),
+              rng.standard_normal((T, 64)).astype(np.float32)):
+        inp["w"] = w
+        up = Uploaded(wl, inp)
+        idx, sc = _run(up, decode=True)
+        _check(up, idx, sc, list(range(T)))
+
+
+def test_edge_decode_row_longer_than_one_cluster_holds():
+    # 150000 keys: beyond what a cluster of 8 CTAs keeps in registers; decode streams it
+    wl = W.scaled(W.decode(), seq_lens=(150000, 5000), q_lens=(1, 1), seed=42)
+    up = Uploaded(wl)
+    idx, sc = _run(up, decode=True)
+    _check(up, idx, sc, [0, 1])
+
+
 def test_edge_empty_batch_and_zero_query_sequences():
     wl = W.scaled(W.prefill(), seq_lens=(40, 10), q_lens=(0, 10), top_k=16)
     up = Uploaded(wl)
