@@ -78,6 +78,7 @@ struct Plan {
   std::vector<int32_t> topk_rows;
   std::vector<TopkClass> classes;
   std::vector<TopkChunk> chunks;     // streaming top-k (then `classes` is empty)
+  int64_t rows_first = 0, rows_count = 0;   // row-streaming top-k: range in topk_rows
   int64_t short_first = 0, short_count = 0;
 };
 
@@ -507,6 +508,22 @@ void plan_topk_stream(const BatchView& v, int top_k, Plan* p) {
   p->short_count = static_cast<int64_t>(p->topk_rows.size());
 }
 
+// Prefill rows: one CTA each in the row-streaming top-k, longest rows first.
+void plan_topk_rows(const BatchView& v, int top_k, Plan* p) {
+  std::vector<int32_t> longs;
+  p->topk_rows.clear();
+  p->classes.clear();
+  p->chunks.clear();
+  for (int64_t r = 0; r < v.total_q; ++r)
+    (p->row_pos[r] + 1 <= top_k ? p->topk_rows : longs).push_back(static_cast<int32_t>(r));
+  p->short_first = 0;
+  p->short_count = static_cast<int64_t>(p->topk_rows.size());
+  std::stable_sort(longs.begin(), longs.end(), [&](int32_t x, int32_t y) { return p->row_pos[x] > p->row_pos[y]; });
+  p->rows_first = p->short_count;
+  p->rows_count = static_cast<int64_t>(longs.size());
+  p->topk_rows.insert(p->topk_rows.end(), longs.begin(), longs.end());
+}
+
 MetaLayout layout_of(const Plan& p) {
   MetaLayout m;
   size_t o = 0;
@@ -608,8 +625,8 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     np.stream_topk = mode == Mode::Decode;
     if (np.stream_topk)
       plan_topk_stream(v, top_k, &np);
-    else if (mode != Mode::Scores && (st = plan_topk(v, top_k, g_sms, &np)) != DSA_OK)
-      return st;
+    else if (mode == Mode::Prefill)
+      plan_topk_rows(v, top_k, &np);
     const MetaLayout nm = layout_of(np);
     const std::vector<uint8_t> blob = pack(np, nm);
     c->meta_valid = false;
@@ -684,6 +701,13 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     s.rows = rows + cl.first;
     s.n_rows = static_cast<int32_t>(cl.count);
     DSA_CUDA_TRY(launch_topk(s, cl.ept, cl.cluster, stream), "top-k launch");
+    ++g_launches;
+  }
+  if (p.rows_count) {
+    TopkArgs s = ta;
+    s.rows = rows + p.rows_first;
+    s.n_rows = static_cast<int32_t>(p.rows_count);
+    DSA_CUDA_TRY(launch_topk_rows(s, stream), "top-k (row-streaming) launch");
     ++g_launches;
   }
   if (!p.chunks.empty()) {

@@ -106,6 +106,8 @@ bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng);
 // Top-k over rows longer than top_k: one cluster of `cluster` CTAs per row,
 // `ept` keys per thread held in registers.
 cudaError_t launch_topk(const TopkArgs& a, int ept, int cluster, cudaStream_t stream);
+// Rows longer than top_k, one CTA per row streaming it in passes (prefill: many rows).
+cudaError_t launch_topk_rows(const TopkArgs& a, cudaStream_t stream);
 // Rows whose coarse histogram the logits epilogue built: one CTA per chunk of kStreamChunk
 // keys, the last CTA of a row finishing the selection inside the threshold bin.
 cudaError_t launch_topk_stream(const TopkArgs& a, cudaStream_t stream);

@@ -685,6 +685,164 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
   if (!ok && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
 }
 
+// ---- row-streaming top-k (prefill: many rows, no histogram from the logits kernel).
+// One CTA per row, several CTAs per SM; the row is streamed from memory in passes of
+// kRowIter keys with the next iteration's loads in flight, nothing held across passes:
+//   pass 1: a shared-memory histogram of the top 12 key bits gives the bin B holding the
+//           k-th largest key, the number of keys above it and the number inside it;
+//   refinement passes (only while B holds more than kRowCap keys and several values):
+//           histogram of B's keys over 2048 sub-bins, B narrows to the sub-bin;
+//   final pass: keys above B go straight to the output (warp-aggregated slot counter),
+//           keys inside B are gathered into shared memory, or, when B is one tied value,
+//           the first `need` of them are written directly;
+//   the gathered keys are resolved with exact shared-memory levels.
+constexpr int kRowThreads = 256;
+constexpr int kRowEPT = 16;                               // keys per thread per iteration
+constexpr int kRowIter = kRowThreads * kRowEPT;
+constexpr int kRowCap = 4096;                             // interval keys gathered in shared memory
+constexpr int kRowShift0 = 20;                            // first level: 4096 bins of the top 12 bits
+constexpr int kRowBins0 = 1 << (32 - kRowShift0);
+constexpr size_t kRowSmemBytes = (kRowBins0 + 2 * kRowCap) * sizeof(uint32_t);
+static_assert(kRowBins0 % kRowThreads == 0 && kBins % kRowThreads == 0, "bins per thread");
+
+__device__ __forceinline__ void row_load(const float* src, int n, int base, float4 (&f)[kRowEPT / 4]) {
+#pragma unroll
+  for (int v = 0; v < kRowEPT / 4; ++v) {
+    const int i = base + (v * kRowThreads + static_cast<int>(threadIdx.x)) * 4;
+    f[v] = i < n ? __ldcs(reinterpret_cast<const float4*>(src + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+__global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs a) {
+  extern __shared__ __align__(16) uint32_t rsm[];
+  uint32_t* hist = rsm;                                   // kRowBins0 (levels >= 1 use the first kBins)
+  uint32_t* cand_key = rsm + kRowBins0;                   // kRowCap
+  int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kRowCap);
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t lvl_bin, lvl_above, lvl_cnt, ctr_a, ctr_b;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int row = a.rows[blockIdx.x];
+  const int n = a.row_pos[row] + 1;                       // n > top_k
+  const float* src = a.scores + a.row_off[row];
+  const uint32_t k = static_cast<uint32_t>(a.top_k);
+  int32_t* oi = a.out_idx + static_cast<int64_t>(row) * a.top_k;
+  float* os = a.out_score + static_cast<int64_t>(row) * a.top_k;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  uint32_t lo = 0u, hi = 0xFFFFFFFFu;                     // interval holding the keys still to choose
+  uint32_t need = k;                                      // keys still to take from [lo, hi]
+  uint32_t cnt = static_cast<uint32_t>(n);                // keys inside [lo, hi]
+  int shift = kRowShift0;
+  grid_dependency_wait();                                 // the scores come from the previous kernel
+  for (int level = 0;; ++level) {
+    const bool final_pass = cnt <= static_cast<uint32_t>(kRowCap) || lo == hi || level >= 4;
+    const int nbins = level == 0 ? kRowBins0 : kBins;
+    if (!final_pass)
+      for (int b = tid; b < nbins; b += kRowThreads) hist[b] = 0u;
+    if (tid == 0) {
+      ctr_a = 0u;
+      ctr_b = 0u;
+      lvl_bin = kNotFound;
+    }
+    __syncthreads();
+    const uint32_t n_sel_above = k - need;                // keys above hi, all selected
+    float4 cur[kRowEPT / 4];
+    row_load(src, n, 0, cur);
+    for (int base = 0; base < n; base += kRowIter) {
+      float4 nxt[kRowEPT / 4];
+      if (base + kRowIter < n) {
+        row_load(src, n, base + kRowIter, nxt);
+      } else {
+#pragma unroll
+        for (int v = 0; v < kRowEPT / 4; ++v) nxt[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int v = 0; v < kRowEPT / 4; ++v) {
+        const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pos = base + (v * kRowThreads + tid) * 4 + e;
+          const bool valid = pos < n;
+          const uint32_t kk = float_to_key(fv[e]);
+          if (!final_pass) {
+            if (valid && kk >= lo && kk <= hi) atomicAdd(&hist[(kk - lo) >> shift], 1u);
+          } else {
+            const bool up = valid && kk > hi;
+            const uint32_t m_up = __ballot_sync(0xffffffffu, up);
+            if (m_up) {
+              uint32_t b0 = 0u;
+              if (lane == __ffs(m_up) - 1) b0 = atomicAdd(&ctr_a, __popc(m_up));
+              b0 = __shfl_sync(0xffffffffu, b0, __ffs(m_up) - 1);
+              const uint32_t slot = b0 + __popc(m_up & lt_mask);
+              if (up && slot < n_sel_above) {
+                oi[slot] = pos;
+                os[slot] = key_to_float(kk);
+              }
+            }
+            if (valid && kk >= lo && kk <= hi) {
+              const uint32_t t = atomicAdd(&ctr_b, 1u);
+              if (lo == hi) {                             // one tied value: any `need` of them
+                if (t < need) {
+                  oi[n_sel_above + t] = pos;
+                  os[n_sel_above + t] = key_to_float(kk);
+                }
+              } else if (t < static_cast<uint32_t>(kRowCap)) {
+                cand_key[t] = kk;
+                cand_idx[t] = pos;
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < kRowEPT / 4; ++v) cur[v] = nxt[v];
+    }
+    __syncthreads();
+    if (final_pass) {
+      bool ok = ctr_a == n_sel_above && ctr_b == cnt;
+      __syncthreads();                                    // every thread has read the counters
+      if (ok && lo != hi) {
+        if (cnt > static_cast<uint32_t>(kRowCap)) {
+          ok = false;                                     // unreachable: four levels resolve 32 bits
+        } else {
+          ok = rank0_select<false, kRowThreads>(cand_key, cand_idx, cnt, lo, hi, need, n_sel_above, oi, os, hist,
+                                                warp_sums, &lvl_bin, &lvl_above, &lvl_cnt, &ctr_a, &ctr_b);
+        }
+      }
+      if (!ok && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+      return;
+    }
+    // the bin of the need-th largest key inside [lo, hi]
+    if (level == 0) {
+      constexpr int PER = kRowBins0 / kRowThreads;
+      uint32_t c[PER];
+#pragma unroll
+      for (int j = 0; j < PER; ++j) c[j] = hist[kRowBins0 - 1 - (tid * PER + j)];
+      find_threshold_bin<PER>(c, kRowBins0 - 1 - tid * PER, need, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt);
+    } else {
+      constexpr int PER = kBins / kRowThreads;
+      uint32_t c[PER];
+#pragma unroll
+      for (int j = 0; j < PER; ++j) c[j] = hist[kBins - 1 - (tid * PER + j)];
+      find_threshold_bin<PER>(c, kBins - 1 - tid * PER, need, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt);
+    }
+    __syncthreads();
+    if (lvl_bin == kNotFound) {
+      if (tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+      return;
+    }
+    const uint32_t nlo = lo + (lvl_bin << shift);
+    const uint32_t width_m1 = (1u << shift) - 1u;
+    hi = (hi - nlo) > width_m1 ? nlo + width_m1 : hi;
+    lo = nlo;
+    need -= lvl_above;
+    cnt = lvl_cnt;
+    const int bits = lo == hi ? 0 : 32 - __clz(hi - lo);
+    shift = bits > 11 ? bits - 11 : 0;
+    __syncthreads();                                      // lvl_* read before the next level resets them
+  }
+}
+
 // Rows whose whole causal history fits in top_k: every position, then -1 / -inf.
 __global__ void __launch_bounds__(256) topk_short_kernel(const TopkArgs a) {
   grid_dependency_wait();                     // the scores come from the previous kernel
@@ -758,6 +916,31 @@ cudaError_t launch_topk_stream(const TopkArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, topk_stream_kernel, a);
+}
+
+cudaError_t launch_topk_rows(const TopkArgs& a, cudaStream_t stream) {
+  if (a.n_rows <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.n_rows), 1, 1);
+  cfg.blockDim = dim3(kRowThreads, 1, 1);
+  cfg.dynamicSmemBytes = kRowSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static unsigned long long configured = 0;   // one bit per device ordinal
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(configured & (1ull << dev))) {
+    e = cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kRowSmemBytes));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured |= 1ull << dev;
+  }
+  return cudaLaunchKernelEx(&cfg, topk_row_kernel, a);
 }
 
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream) {
