@@ -109,7 +109,8 @@ __device__ __forceinline__ void find_threshold_bin(const uint32_t (&cnt)[PER], u
   }
 }
 
-// Calls f(key, index) for candidates [0, m), each thread taking every NT-th one.  Reads
+// Calls f(key, index, valid) for candidates [0, m), each thread taking every NT-th one
+// (valid is false past m).  Reads
 // go in batches of CPT per thread, all loads of a batch issued before any is used: global
 // candidates cost an L2 round trip each, which a one-at-a-time loop would serialise.
 template <bool kGlobal, bool kWithIdx, int NT, int CPT, class F>
@@ -128,20 +129,20 @@ __device__ __forceinline__ void for_candidates(const uint32_t* ck, const int32_t
       }
     }
 #pragma unroll
-    for (int j = 0; j < CPT; ++j)
-      if (b0 + j * NT + threadIdx.x < m) f(kk[j], ix[j]);
+    for (int j = 0; j < CPT; ++j) f(kk[j], ix[j], b0 + j * NT + threadIdx.x < m);
   }
 }
 
-// One CTA, all its threads: among the m gathered keys in [lo, hi] (candidates in this
-// CTA's shared memory, or with kGlobalCand in global memory, read through the L2 since
-// other CTAs wrote them), write the `need` largest to slots [base, base + need) of the row.
+// One CTA, all its threads: the m gathered keys (in this CTA's shared memory, or with
+// kGlobalCand in global memory, read through the L2 since other CTAs wrote them) are
+// n_up keys above hi, all selected, and m - n_up keys in [lo, hi] of which the `need`
+// largest are selected; all n_up + need go to slots [base, base + n_up + need) of the row.
 // Exact: CTA-local histogram levels narrow [lo, hi] by >= 2^10 per level; keys above the
 // final interval are taken, then `need` of its keys (a single tied value if not resolved).
 // Returns false if the counts turn out inconsistent (nothing is written past the row).
 template <bool kGlobalCand, int NT>
-__device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, uint32_t m, uint32_t lo,
-                             uint32_t hi, uint32_t need, uint32_t base, int32_t* oi, float* os, uint32_t* hist,
+__device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, uint32_t m, uint32_t n_up,
+                             uint32_t lo, uint32_t hi, uint32_t need, uint32_t base, int32_t* oi, float* os, uint32_t* hist,
                              uint32_t* warp_sums, uint32_t* lvl_bin, uint32_t* lvl_above, uint32_t* lvl_cnt,
                              uint32_t* ctr_a, uint32_t* ctr_b) {
   constexpr int PER = kBins / NT;
@@ -151,15 +152,15 @@ __device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, 
   ls.lo = lo;
   ls.hi = hi;
   ls.need = need;
-  ls.done = need == m ? 1u : 0u;
+  ls.done = need == m - n_up ? 1u : 0u;
   for (int level = 0; level < 4 && !ls.done; ++level) {
     if (ls.lo == ls.hi) { ls.done = 2; break; }
     const int bits = 32 - __clz(ls.hi - ls.lo);
     const int shift = bits > 11 ? bits - 11 : 0;
     for (int b = tid; b < kBins; b += NT) hist[b] = 0u;
     __syncthreads();
-    for_candidates<kGlobalCand, false, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t) {
-      if (kk >= ls.lo && kk <= ls.hi) atomicAdd(&hist[(kk - ls.lo) >> shift], 1u);
+    for_candidates<kGlobalCand, false, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t, bool valid) {
+      if (valid && kk >= ls.lo && kk <= ls.hi) atomicAdd(&hist[(kk - ls.lo) >> shift], 1u);
     });
     __syncthreads();
     uint32_t c[PER];
@@ -184,8 +185,10 @@ __device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, 
     *ctr_b = 0u;
   }
   __syncthreads();
-  const uint32_t first_in = base + (need - ls.need);     // slots of interval keys start here
-  for_candidates<kGlobalCand, true, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t ix) {
+  const uint32_t n_sel_up = n_up + (need - ls.need);     // keys above the final interval
+  const uint32_t first_in = base + n_sel_up;             // slots of interval keys start here
+  for_candidates<kGlobalCand, true, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t ix, bool valid) {
+    if (!valid) return;
     if (kk > ls.hi) {
       const uint32_t slot = base + atomicAdd(ctr_a, 1u);
       if (slot < first_in) {
@@ -201,7 +204,7 @@ __device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, 
     }
   });
   __syncthreads();
-  return *ctr_a == need - ls.need && *ctr_b >= ls.need && !(ls.done == 1 && *ctr_b != ls.need);
+  return *ctr_a == n_sel_up && *ctr_b >= ls.need && !(ls.done == 1 && *ctr_b != ls.need);
 }
 
 template <int EPT>
@@ -381,7 +384,7 @@ topk_kernel(const TopkArgs a) {
     cluster.sync();                           // rank 0 holds the whole bin; counters are final
     if (crank != 0) return;                   // nobody reads another CTA's memory after this point
     const bool above_ok = cnt_above == n_above_total && cnt_cand == bcount;
-    const bool ok = rank0_select<false, kThreads>(cand_key, cand_idx, bcount, bin_lo, bin_hi, need0, n_above_total, oi, os, hist,
+    const bool ok = rank0_select<false, kThreads>(cand_key, cand_idx, bcount, 0u, bin_lo, bin_hi, need0, n_above_total, oi, os, hist,
                                  warp_sums, &lvl_bin, &lvl_above, &lvl_cnt, &base_above, &base_cand);
     if ((!ok || !above_ok) && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
     return;
@@ -655,7 +658,8 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
     }
     __syncthreads();
     for_candidates<true, true, kStreamThreads, 8>(a.cand_key + off, a.cand_idx + off, bcount,
-                                                   [&](uint32_t kk, int32_t ix) {
+                                                   [&](uint32_t kk, int32_t ix, bool valid) {
+      if (!valid) return;
       if (kk > sub_hi) {
         const uint32_t t = atomicAdd(&ctr_a, 1u);
         if (t < above1) {
@@ -673,12 +677,12 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
     __syncthreads();
     const bool pass_ok = ctr_a == above1 && ctr_b == cnt1;
     __syncthreads();                          // every thread has read the counters
-    ok = pass_ok && rank0_select<false, kStreamThreads>(sub_key, sub_idx, cnt1, sub_lo, sub_hi, need0 - above1,
+    ok = pass_ok && rank0_select<false, kStreamThreads>(sub_key, sub_idx, cnt1, 0u, sub_lo, sub_hi, need0 - above1,
                                                          n_above_total + above1, oi, os, hist, warp_sums, &lvl_bin,
                                                          &lvl_above, &lvl_cnt, &ctr_a, &ctr_b);
   } else {
     // a crowded sub-bin (many equal scores): refine over all the row's candidates
-    ok = rank0_select<true, kStreamThreads>(a.cand_key + off, a.cand_idx + off, bcount, bin_lo, bin_hi, need0,
+    ok = rank0_select<true, kStreamThreads>(a.cand_key + off, a.cand_idx + off, bcount, 0u, bin_lo, bin_hi, need0,
                                             n_above_total, oi, os, hist, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt,
                                             &ctr_a, &ctr_b);
   }
@@ -692,9 +696,12 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
 //           k-th largest key, the number of keys above it and the number inside it;
 //   refinement passes (only while B holds more than kRowCap keys and several values):
 //           histogram of B's keys over 2048 sub-bins, B narrows to the sub-bin;
-//   final pass: keys above B go straight to the output (warp-aggregated slot counter),
-//           keys inside B are gathered into shared memory, or, when B is one tied value,
-//           the first `need` of them are written directly;
+//   final pass: when the keys above B and inside B fit in shared memory together (the
+//           usual case), every key >= B's lower edge is gathered there; otherwise keys
+//           above B go straight to the output and B's keys are gathered, or, when B is one
+//           tied value, the first `need` of them are written directly; slots come from a
+//           warp scan of the per-thread counts and one 64-bit shared atomic per warp and
+//           iteration (direct writes: high word, gathered: low word);
 //   the gathered keys are resolved with exact shared-memory levels.
 constexpr int kRowThreads = 256;
 constexpr int kRowEPT = 16;                               // keys per thread per iteration
@@ -720,6 +727,7 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
   int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kRowCap);
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t lvl_bin, lvl_above, lvl_cnt, ctr_a, ctr_b;
+  __shared__ unsigned long long slot_ctr;
   const int tid = threadIdx.x, lane = tid & 31;
   const int row = a.rows[blockIdx.x];
   const int n = a.row_pos[row] + 1;                       // n > top_k
@@ -727,7 +735,6 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
   const uint32_t k = static_cast<uint32_t>(a.top_k);
   int32_t* oi = a.out_idx + static_cast<int64_t>(row) * a.top_k;
   float* os = a.out_score + static_cast<int64_t>(row) * a.top_k;
-  const uint32_t lt_mask = (1u << lane) - 1u;
 
   uint32_t lo = 0u, hi = 0xFFFFFFFFu;                     // interval holding the keys still to choose
   uint32_t need = k;                                      // keys still to take from [lo, hi]
@@ -740,12 +747,12 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
     if (!final_pass)
       for (int b = tid; b < nbins; b += kRowThreads) hist[b] = 0u;
     if (tid == 0) {
-      ctr_a = 0u;
-      ctr_b = 0u;
+      slot_ctr = 0ull;
       lvl_bin = kNotFound;
     }
     __syncthreads();
     const uint32_t n_sel_above = k - need;                // keys above hi, all selected
+    const bool gather_all = n_sel_above + cnt <= static_cast<uint32_t>(kRowCap);
     float4 cur[kRowEPT / 4];
     row_load(src, n, 0, cur);
     for (int base = 0; base < n; base += kRowIter) {
@@ -756,40 +763,65 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
 #pragma unroll
         for (int v = 0; v < kRowEPT / 4; ++v) nxt[v] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      if (!final_pass) {
 #pragma unroll
-      for (int v = 0; v < kRowEPT / 4; ++v) {
-        const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+        for (int v = 0; v < kRowEPT / 4; ++v) {
+          const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int pos = base + (v * kRowThreads + tid) * 4 + e;
-          const bool valid = pos < n;
-          const uint32_t kk = float_to_key(fv[e]);
-          if (!final_pass) {
-            if (valid && kk >= lo && kk <= hi) atomicAdd(&hist[(kk - lo) >> shift], 1u);
-          } else {
-            const bool up = valid && kk > hi;
-            const uint32_t m_up = __ballot_sync(0xffffffffu, up);
-            if (m_up) {
-              uint32_t b0 = 0u;
-              if (lane == __ffs(m_up) - 1) b0 = atomicAdd(&ctr_a, __popc(m_up));
-              b0 = __shfl_sync(0xffffffffu, b0, __ffs(m_up) - 1);
-              const uint32_t slot = b0 + __popc(m_up & lt_mask);
-              if (up && slot < n_sel_above) {
-                oi[slot] = pos;
-                os[slot] = key_to_float(kk);
+          for (int e = 0; e < 4; ++e) {
+            const int pos = base + (v * kRowThreads + tid) * 4 + e;
+            const uint32_t kk = float_to_key(fv[e]);
+            if (pos < n && kk >= lo && kk <= hi) atomicAdd(&hist[(kk - lo) >> shift], 1u);
+          }
+        }
+      } else {
+        uint32_t up_mask = 0u, in_mask = 0u;              // bit j: key j is above / inside [lo, hi]
+#pragma unroll
+        for (int v = 0; v < kRowEPT / 4; ++v) {
+          const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool valid = base + (v * kRowThreads + tid) * 4 + e < n;
+            const uint32_t kk = float_to_key(fv[e]);
+            up_mask |= static_cast<uint32_t>(!gather_all && valid && kk > hi) << (v * 4 + e);
+            in_mask |= static_cast<uint32_t>(valid && kk >= lo && (gather_all || kk <= hi)) << (v * 4 + e);
+          }
+        }
+        const unsigned long long mine = (static_cast<unsigned long long>(__popc(up_mask)) << 32) | __popc(in_mask);
+        unsigned long long incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        unsigned long long wbase = 0ull;
+        if (lane == 31 && incl) wbase = atomicAdd(&slot_ctr, incl);
+        wbase = __shfl_sync(0xffffffffu, wbase, 31) + (incl - mine);
+        uint32_t iu = static_cast<uint32_t>(wbase >> 32), ic = static_cast<uint32_t>(wbase);
+#pragma unroll
+        for (int v = 0; v < kRowEPT / 4; ++v) {
+          const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t kk = float_to_key(fv[e]);
+            const int pos = base + (v * kRowThreads + tid) * 4 + e;
+            if ((up_mask >> (v * 4 + e)) & 1u) {
+              if (iu < n_sel_above) {
+                oi[iu] = pos;
+                os[iu] = key_to_float(kk);
               }
-            }
-            if (valid && kk >= lo && kk <= hi) {
-              const uint32_t t = atomicAdd(&ctr_b, 1u);
-              if (lo == hi) {                             // one tied value: any `need` of them
-                if (t < need) {
-                  oi[n_sel_above + t] = pos;
-                  os[n_sel_above + t] = key_to_float(kk);
+              ++iu;
+            } else if ((in_mask >> (v * 4 + e)) & 1u) {
+              if (lo == hi && !gather_all) {              // one tied value: any `need` of them
+                if (ic < need) {
+                  oi[n_sel_above + ic] = pos;
+                  os[n_sel_above + ic] = key_to_float(kk);
                 }
-              } else if (t < static_cast<uint32_t>(kRowCap)) {
-                cand_key[t] = kk;
-                cand_idx[t] = pos;
+              } else if (ic < static_cast<uint32_t>(kRowCap)) {
+                cand_key[ic] = kk;
+                cand_idx[ic] = pos;
               }
+              ++ic;
             }
           }
         }
@@ -799,14 +831,16 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
     }
     __syncthreads();
     if (final_pass) {
-      bool ok = ctr_a == n_sel_above && ctr_b == cnt;
+      const uint32_t direct = gather_all ? 0u : n_sel_above, gathered = gather_all ? n_sel_above + cnt : cnt;
+      bool ok = static_cast<uint32_t>(slot_ctr >> 32) == direct && static_cast<uint32_t>(slot_ctr) == gathered;
       __syncthreads();                                    // every thread has read the counters
-      if (ok && lo != hi) {
-        if (cnt > static_cast<uint32_t>(kRowCap)) {
+      if (ok && (gather_all || lo != hi)) {
+        if (gathered > static_cast<uint32_t>(kRowCap)) {
           ok = false;                                     // unreachable: four levels resolve 32 bits
         } else {
-          ok = rank0_select<false, kRowThreads>(cand_key, cand_idx, cnt, lo, hi, need, n_sel_above, oi, os, hist,
-                                                warp_sums, &lvl_bin, &lvl_above, &lvl_cnt, &ctr_a, &ctr_b);
+          ok = rank0_select<false, kRowThreads>(cand_key, cand_idx, gathered, n_sel_above - direct, lo, hi, need,
+                                                direct, oi, os, hist, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt,
+                                                &ctr_a, &ctr_b);
         }
       }
       if (!ok && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);

@@ -235,6 +235,24 @@ def test_edge_ties_and_zero_and_negative_weights():
         _check(up, idx, sc, [0, 1, 99, 100, 101, 500, 1499])
 
 
+def test_edge_prefill_ties_in_rows_longer_than_the_gather_buffer():
+    # rows of up to 9000 keys with few distinct scores: the threshold bin holds more keys
+    # than one CTA gathers, so the row top-k refines it, or (zero weights: one tied value)
+    # writes the tied keys directly
+    L = 9000
+    wl = W.scaled(W.prefill(), seq_lens=(L,), q_lens=(L,), outlier_frac=0.0, seed=43)
+    inp = W.make_inputs(wl)
+    rng = np.random.default_rng(3)
+    inp["k_bits"] = [W.f32_to_bf16_bits(rng.integers(-2, 3, (L, 128)).astype(np.float32))]
+    inp["q_bits"] = W.f32_to_bf16_bits(rng.integers(-1, 2, (L, 64, 128)).astype(np.float32))
+    rows = [0, 2047, 2048, 4095, 4096, 4097, 6000, L - 1]
+    for w in (np.full((L, 64), 1.0 / 64, np.float32), np.zeros((L, 64), np.float32)):
+        inp["w"] = w
+        up = Uploaded(wl, inp)
+        idx, sc = _run(up)
+        _check(up, idx, sc, rows)
+
+
 def test_edge_decode_ties_zero_and_negative_weights():
     # decode rows over several chunks of the streaming top-k; with zero weights every
     # score is 0, so the threshold bin holds the whole row and the choice is all ties
