@@ -58,6 +58,9 @@ def parse():
                     help="decode (the default) is the measured workload; the others are for profiling")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="profiling only: run a prefill workload at this sequence length instead")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="profiling only: run this many untimed steps of the workload and exit (no JSON line); "
+                         "the command ncu wraps to capture single kernels")
     return ap.parse_args()
 
 
@@ -368,6 +371,15 @@ def run_ours(args):
         wl = W.scaled(wl, seq_lens=(args.seq_len,), q_lens=(args.seq_len,))
     inp = host_inputs(wl)
     hx = Harness(wl, inp, dev, stream)
+
+    if args.profile_steps > 0:
+        with torch.cuda.stream(stream):
+            for _ in range(args.profile_steps):
+                hx.step()
+        api.dsa_check_device_errors(stream)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     # uncaptured warm-up (also plans the batch once)
     with torch.cuda.stream(stream):
