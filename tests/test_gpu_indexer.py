@@ -184,8 +184,9 @@ def test_decode_bf16_ragged(q_len):
     _check(up, idx, sc, list(range(wl.total_q)))
 
 
-def test_decode_fp8_ragged_pairs():
-    wl = W.scaled(W.decode8(), seq_lens=(9000, 2049, 4097, 3000, 2), q_lens=(2,) * 5)
+@pytest.mark.parametrize("q_len", [1, 2, 3])
+def test_decode_fp8_ragged(q_len):
+    wl = W.scaled(W.decode8(), seq_lens=(9000, 2049, 4097, 3000, 3), q_lens=(q_len,) * 5, seed=20 + q_len)
     up = Uploaded(wl)
     idx, sc = _run(up, decode=True)
     _check(up, idx, sc, list(range(wl.total_q)))
