@@ -691,7 +691,13 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
 
 // ---- row-streaming top-k (prefill: many rows, no histogram from the logits kernel).
 // One CTA per row, several CTAs per SM; the row is streamed from memory in passes of
-// kRowIter keys with the next iteration's loads in flight, nothing held across passes:
+// kRowIter keys with the next iteration's loads in flight, nothing held across passes.
+// Sampled first try (rows longer than kRowCap): one key in 16 (a float4 per 64 keys) is
+// read into shared memory; a histogram over the sample's own key range gives a threshold
+// tau expected to leave about 1.25 k + 64 keys at or above it; one pass with one float
+// compare per key gathers those keys into shared memory, and if there are between k and
+// kRowCap of them the exact select runs on that set (the k largest keys of the row are all
+// >= tau whenever at least k keys are).  Otherwise, and for rows it does not apply to:
 //   pass 1: a shared-memory histogram of the top 12 key bits gives the bin B holding the
 //           k-th largest key, the number of keys above it and the number inside it;
 //   refinement passes (only while B holds more than kRowCap keys and several values):
@@ -720,13 +726,162 @@ __device__ __forceinline__ void row_load(const float* src, int n, int base, floa
   }
 }
 
+// The sampled first try described above; returns true when it handled the row (a broken
+// count invariant is recorded in *err).  All threads of the CTA call it and get the same
+// answer; on false nothing has been written.
+__device__ bool row_sampled_select(const float* src, int n, uint32_t k, int32_t* oi, float* os, uint32_t* hist,
+                                   uint32_t* cand_key, int32_t* cand_idx, uint32_t* warp_sums, uint32_t* lvl_bin,
+                                   uint32_t* lvl_above, uint32_t* lvl_cnt, uint32_t* ctr_a, uint32_t* ctr_b,
+                                   uint32_t* ctr_c, int* err, int row) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  // ---- sample: the first float4 of every `block` keys (block a multiple of 64, s <= kRowCap)
+  const int block = 64 * ((n + 65535) / 65536);
+  const int n_blocks = (n + block - 1) / block;
+  uint32_t smin = 0xFFFFFFFFu, smax = 0u, s_local = 0u;
+  for (int b = tid; b < n_blocks; b += kRowThreads) {
+    const int i = b * block;
+    const float4 f = __ldcs(reinterpret_cast<const float4*>(src + i));
+    const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool valid = i + e < n;
+      const uint32_t kk = float_to_key(fv[e]);
+      cand_key[4 * b + e] = valid ? kk : 0u;
+      if (valid) {
+        smin = min(smin, kk);
+        smax = max(smax, kk);
+        ++s_local;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    smin = min(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+    smax = max(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+  }
+  if (tid == 0) {
+    *ctr_a = 0xFFFFFFFFu;                     // sample min
+    *ctr_b = 0u;                              // sample max
+  }
+  for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0u;
+  uint32_t s_valid;
+  block_exclusive_scan(s_local, warp_sums, s_valid);       // also orders the resets above
+  if (lane == 0) {
+    atomicMin(ctr_a, smin);
+    atomicMax(ctr_b, smax);
+  }
+  __syncthreads();
+  const uint32_t lo_s = *ctr_a, hi_s = *ctr_b;
+  const int bits = hi_s > lo_s ? 32 - __clz(hi_s - lo_s) : 0;
+  const int shift = bits > 11 ? bits - 11 : 0;
+  for (int i = tid; i < 4 * n_blocks; i += kRowThreads) {
+    const uint32_t kk = cand_key[i];
+    if (i < 4 * n_blocks && ((i & 3) + (i >> 2) * block) < n) atomicAdd(&hist[(kk - lo_s) >> shift], 1u);
+  }
+  // sample rank of tau: about (1.25 k + 64) keys of the row expected at or above it
+  const uint32_t r = static_cast<uint32_t>(
+      (static_cast<unsigned long long>(k + k / 4 + 64) * s_valid + static_cast<unsigned long long>(n) - 1) /
+      static_cast<unsigned long long>(n));
+  if (tid == 0) *lvl_bin = kNotFound;
+  {
+    constexpr int PER = kBins / kRowThreads;
+    uint32_t c[PER];
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < PER; ++j) c[j] = hist[kBins - 1 - (tid * PER + j)];
+    find_threshold_bin<PER>(c, kBins - 1 - tid * PER, r, warp_sums, lvl_bin, lvl_above, lvl_cnt);
+  }
+  __syncthreads();
+  if (*lvl_bin == kNotFound) return false;    // the sample holds fewer than r keys
+  const uint32_t tau = lo_s + (*lvl_bin << shift);
+  const float tau_f = key_to_float(tau);
+  if (tid == 0) {
+    *ctr_a = 0u;                              // gathered keys
+    *ctr_b = 0u;                              // largest gathered key
+    *ctr_c = 0xFFFFFFFFu;                     // smallest gathered key
+  }
+  __syncthreads();
+
+  // ---- one pass: every key >= tau into shared memory (slots: warp scan + one atomic per warp).
+  // {f >= tau_f} is closed upwards in key order (key order refines float order), so it holds
+  // the k largest keys as soon as it has k elements.
+  uint32_t my_max = 0u, my_min = 0xFFFFFFFFu;
+  float4 cur[kRowEPT / 4];
+  row_load(src, n, 0, cur);
+  for (int base = 0; base < n; base += kRowIter) {
+    float4 nxt[kRowEPT / 4];
+    if (base + kRowIter < n) {
+      row_load(src, n, base + kRowIter, nxt);
+    } else {
+#pragma unroll
+      for (int v = 0; v < kRowEPT / 4; ++v) nxt[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    uint32_t sel = 0u;
+#pragma unroll
+    for (int v = 0; v < kRowEPT / 4; ++v) {
+      const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        sel |= static_cast<uint32_t>(fv[e] >= tau_f && base + (v * kRowThreads + tid) * 4 + e < n) << (v * 4 + e);
+    }
+    const uint32_t mine = __popc(sel);
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t wbase = 0u;
+    if (lane == 31 && incl) wbase = atomicAdd(ctr_a, incl);
+    uint32_t slot = __shfl_sync(0xffffffffu, wbase, 31) + incl - mine;
+    if (sel) {
+#pragma unroll
+      for (int v = 0; v < kRowEPT / 4; ++v) {
+        const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((sel >> (v * 4 + e)) & 1u) {
+            const uint32_t kk = float_to_key(fv[e]);
+            my_max = max(my_max, kk);
+            my_min = min(my_min, kk);
+            if (slot < static_cast<uint32_t>(kRowCap)) {
+              cand_key[slot] = kk;
+              cand_idx[slot] = base + (v * kRowThreads + tid) * 4 + e;
+            }
+            ++slot;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < kRowEPT / 4; ++v) cur[v] = nxt[v];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
+    my_min = min(my_min, __shfl_xor_sync(0xffffffffu, my_min, o));
+  }
+  if (lane == 0 && my_max) {
+    atomicMax(ctr_b, my_max);
+    atomicMin(ctr_c, my_min);
+  }
+  __syncthreads();
+  const uint32_t c = *ctr_a, kmax = *ctr_b, kmin = *ctr_c;
+  __syncthreads();                            // every thread has read the counters
+  if (c < k || c > static_cast<uint32_t>(kRowCap)) return false;   // tau missed: exact passes instead
+  const bool ok = rank0_select<false, kRowThreads>(cand_key, cand_idx, c, 0u, kmin, kmax, k, 0u, oi, os, hist,
+                                                   warp_sums, lvl_bin, lvl_above, lvl_cnt, ctr_a, ctr_b);
+  if (!ok && tid == 0) record_error(err, DSA_DEVERR_TOPK, row);
+  return true;
+}
+
 __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint32_t rsm[];
   uint32_t* hist = rsm;                                   // kRowBins0 (levels >= 1 use the first kBins)
   uint32_t* cand_key = rsm + kRowBins0;                   // kRowCap
   int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kRowCap);
   __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t lvl_bin, lvl_above, lvl_cnt, ctr_a, ctr_b;
+  __shared__ uint32_t lvl_bin, lvl_above, lvl_cnt, ctr_a, ctr_b, ctr_c;
   __shared__ unsigned long long slot_ctr;
   const int tid = threadIdx.x, lane = tid & 31;
   const int row = a.rows[blockIdx.x];
@@ -741,6 +896,10 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
   uint32_t cnt = static_cast<uint32_t>(n);                // keys inside [lo, hi]
   int shift = kRowShift0;
   grid_dependency_wait();                                 // the scores come from the previous kernel
+  if (n > kRowCap && k <= static_cast<uint32_t>(kRowCap) / 2 &&
+      row_sampled_select(src, n, k, oi, os, hist, cand_key, cand_idx, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt,
+                         &ctr_a, &ctr_b, &ctr_c, a.err, row))
+    return;
   for (int level = 0;; ++level) {
     const bool final_pass = cnt <= static_cast<uint32_t>(kRowCap) || lo == hi || level >= 4;
     const int nbins = level == 0 ? kRowBins0 : kBins;
