@@ -157,6 +157,30 @@ DSA_API dsa_status_t dsa_indexer_decode(const dsa_query_t* q, const dsa_kcache_t
                                 void* stream);
 
 /*
+ * One whole decode step from host memory (the serving loop of the second page, §2: append
+ * the new token's key, score it and the cache, select), enqueued on `stream` without
+ * waiting for it:
+ *   1. copies k_new_host [n_new, d_I] (k_new_dtype: DSA_BF16 or DSA_F32) and
+ *      dst_rows_host [n_new] to the device and appends them as dsa_indexer_kcache_append;
+ *   2. copies q->data [T, H_I, d_I] (q->dtype), q->scale [T] (FP8) and w_host [T, H_I]
+ *      to the device and scores + selects as dsa_indexer_decode (T = sum of q_lens);
+ *      bf16 queries against an FP8 cache are first quantised on the device as
+ *      dsa_quantize_rows_fp8 does (one scale per token);
+ *   3. copies the selection back into out_idx_host / out_score_host [T, top_k].
+ * Here q->data and q->scale are HOST pointers, like every *_host argument.  Page-locked
+ * host memory keeps the copies asynchronous; pageable memory works, with CUDA staging it.
+ * The device copies live in library-owned buffers of `stream`, reused by the next call on
+ * that stream (stream order makes this safe); the host outputs are complete once the
+ * stream has finished (e.g. dsa_check_device_errors).  n_new may be 0.  Not capturable in
+ * a CUDA graph (DSA_ERR_UNSUPPORTED while `stream` is capturing).
+ */
+DSA_API dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                             const void* k_new_host, dsa_dtype_t k_new_dtype,
+                                             const int64_t* dst_rows_host, int32_t n_new, const dsa_batch_t* batch,
+                                             int32_t top_k, int32_t* out_idx_host, float* out_score_host,
+                                             void* stream);
+
+/*
  * The scores alone, without selection (the first page's index_scores, §3):
  * out_scores[r * ld + s] = I[p_r, s] for s = 0..p_r.  Entries with s > p_r are
  * not written.  ld >= max(seq_lens) and ld % 4 == 0.

@@ -24,6 +24,7 @@ EXPORTED = (
     "dsa_indexer_prefill",
     "dsa_indexer_decode",
     "dsa_indexer_decode_noalloc",
+    "dsa_indexer_decode_host",
     "dsa_indexer_scores",
     "dsa_indexer_workspace_bytes",
     "dsa_set_workspace",
@@ -80,6 +81,8 @@ def load() -> ctypes.CDLL:
         fn.restype = st
     lib.dsa_indexer_decode_noalloc.argtypes = [P(Query), P(KCache), V, P(Batch), I32, V, V, V, V]
     lib.dsa_indexer_decode_noalloc.restype = st
+    lib.dsa_indexer_decode_host.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V, V]
+    lib.dsa_indexer_decode_host.restype = st
     lib.dsa_indexer_scores.argtypes = [P(Query), P(KCache), V, P(Batch), V, I64, V]
     lib.dsa_indexer_scores.restype = st
     lib.dsa_indexer_workspace_bytes.argtypes = [P(Query), P(Batch), I32]

@@ -169,6 +169,34 @@ def dsa_indexer_decode_noalloc(q, cache: IndexerKCache, w, seq_lens, q_lens, top
     return out_idx, out_score
 
 
+def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: IndexerKCache, seq_lens, q_lens,
+                            top_k, out_idx_host, out_score_host, q_scale_host=None, k_base=None, stream=None):
+    """One decode step from HOST tensors in a single library call (dsa_indexer_decode_host):
+    upload the new keys (bf16 or fp32 [n_new, d_I], cache rows ``dst_rows_host`` int64), queries
+    [T, H_I, d_I] (bf16, or uint8 E4M3 codes with ``q_scale_host``) and weights [T, H_I] fp32,
+    append, score + select, and copy the selection into ``out_idx_host`` int32 / ``out_score_host``
+    fp32 [T, top_k].  Returns at once; the host outputs are complete when ``stream`` has finished.
+    Pinned host tensors keep the copies asynchronous."""
+    for t in (q_host, w_host, k_new_host, dst_rows_host, out_idx_host, out_score_host, q_scale_host):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("dsa_indexer_decode_host takes contiguous host tensors")
+    if w_host.dtype != torch.float32 or out_score_host.dtype != torch.float32 or out_idx_host.dtype != torch.int32:
+        raise TypeError("w and out_score must be fp32, out_idx int32")
+    if dst_rows_host.dtype != torch.int64:
+        raise TypeError("dst_rows must be int64")
+    if q_host.dim() != 3:
+        raise ValueError("q must be [T_total, H_I, d_I]")
+    b = _HostBatch(seq_lens, q_lens, k_base)
+    qq = Query(q_host.data_ptr(), q_scale_host.data_ptr() if q_scale_host is not None else None, _dtype_code(q_host),
+               q_host.shape[1], q_host.shape[2])
+    kc = cache.c()
+    n_new = int(k_new_host.shape[0]) if k_new_host is not None else 0
+    check(_lib.load().dsa_indexer_decode_host(ctypes.byref(qq), ctypes.byref(kc), _ptr(w_host), _ptr(k_new_host),
+                                              _dtype_code(k_new_host) if n_new else DSA_BF16, _ptr(dst_rows_host),
+                                              n_new, ctypes.byref(b.c), top_k, _ptr(out_idx_host),
+                                              _ptr(out_score_host), _stream(stream)))
+
+
 def dsa_indexer_scores(q, cache: IndexerKCache, w, seq_lens, q_scale=None, q_lens=None, k_base=None, ld=None,
                        out=None, stream=None):
     """Dense scores [T_total, ld] (entries after each query's position are left as they were: -inf here)."""

@@ -140,6 +140,8 @@ struct Ctx {
   MetaLayout layout;
   void* cur_meta = nullptr;       // tables of the cached plan
   float* cur_scores = nullptr;    // score workspace of the cached plan
+  void* d_host_stage = nullptr;   // dsa_indexer_decode_host: device copies of the step's inputs/outputs
+  size_t host_stage_cap = 0;
 };
 
 std::mutex g_mu;
@@ -799,6 +801,91 @@ dsa_status_t dsa_indexer_decode(const dsa_query_t* q, const dsa_kcache_t* kc, co
                                 const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx, float* out_score,
                                 void* stream) {
   return run_indexer(Mode::Decode, q, kc, w, batch, top_k, out_idx, out_score, nullptr, 0, stream);
+}
+
+dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                     const void* k_new_host, dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host,
+                                     int32_t n_new, const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
+                                     float* out_score_host, void* stream_v) {
+  g_last_error.clear();
+  dsa_status_t st = check_cache(kc);
+  if (st != DSA_OK) return st;
+  if (!q || !batch || !w_host || !out_idx_host || !out_score_host || !q->data)
+    return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (n_new < 0 || (n_new > 0 && (!k_new_host || !dst_rows_host)))
+    return fail(DSA_ERR_INVALID_ARG, "n_new < 0, or k_new_host / dst_rows_host is NULL");
+  if (k_new_dtype != DSA_BF16 && k_new_dtype != DSA_F32) return fail(DSA_ERR_INVALID_ARG, "k_new_dtype must be DSA_BF16 or DSA_F32");
+  if (q->dtype != DSA_BF16 && q->dtype != DSA_FP8_E4M3) return fail(DSA_ERR_INVALID_ARG, "q->dtype must be DSA_BF16 or DSA_FP8_E4M3");
+  if (q->dtype == DSA_FP8_E4M3 && !q->scale) return fail(DSA_ERR_INVALID_ARG, "FP8 queries need q->scale");
+  // bf16 queries against an FP8 cache are quantised on the device after the upload
+  const bool quantise_q = q->dtype == DSA_BF16 && kc->dtype == DSA_FP8_E4M3;
+  if (q->H_I <= 0 || q->d_I <= 0 || top_k <= 0) return fail(DSA_ERR_INVALID_ARG, "H_I, d_I and top_k must be positive");
+  if (batch->num_seqs < 0 || (batch->num_seqs > 0 && (!batch->seq_lens || !batch->q_lens)))
+    return fail(DSA_ERR_INVALID_ARG, "decode needs batch.seq_lens and batch.q_lens");
+  int64_t T = 0;
+  for (int i = 0; i < batch->num_seqs; ++i) T += batch->q_lens[i];
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  DSA_CUDA_TRY(cudaStreamIsCapturing(stream, &cap), "cudaStreamIsCapturing");
+  if (cap != cudaStreamCaptureStatusNone) return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_decode_host cannot be captured");
+  Ctx* c = nullptr;
+  if ((st = get_ctx(stream, &c)) != DSA_OK) return st;
+
+  // device staging: [k_new | dst_rows | q | q_scale | w | out_idx | out_score | q8 | q8_scale],
+  // 256-byte aligned parts (the last two only when bf16 queries meet an FP8 cache)
+  const size_t esz_k = k_new_dtype == DSA_F32 ? 4 : 2, esz_q = q->dtype == DSA_FP8_E4M3 ? 1 : 2;
+  const size_t q_elems = size_t(T) * q->H_I * q->d_I;
+  const size_t b_k = size_t(n_new) * kc->d_I * esz_k, b_rows = size_t(n_new) * sizeof(int64_t);
+  const size_t b_q = q_elems * esz_q, b_qs = q->dtype == DSA_FP8_E4M3 ? size_t(T) * 4 : 0;
+  const size_t b_w = size_t(T) * q->H_I * 4, b_out = size_t(T) * top_k * 4;
+  const size_t o_rows = align_up(b_k), o_q = o_rows + align_up(b_rows), o_qs = o_q + align_up(b_q);
+  const size_t o_w = o_qs + align_up(b_qs), o_oi = o_w + align_up(b_w), o_os = o_oi + align_up(b_out);
+  const size_t o_q8 = o_os + align_up(b_out), o_q8s = o_q8 + (quantise_q ? align_up(q_elems) : 0);
+  const size_t total = o_q8s + (quantise_q ? align_up(size_t(T) * 4) : 0);
+  if (total > c->host_stage_cap) {
+    if (c->d_host_stage) {
+      DSA_CUDA_TRY(cudaStreamSynchronize(stream), "cudaStreamSynchronize");   // earlier calls may still read it
+      DSA_CUDA_TRY(cudaFree(c->d_host_stage), "cudaFree");
+      c->d_host_stage = nullptr;
+      c->host_stage_cap = 0;
+    }
+    DSA_CUDA_TRY(cudaMalloc(&c->d_host_stage, total), "cudaMalloc(host-step staging)");
+    c->host_stage_cap = total;
+  }
+  char* d = static_cast<char*>(c->d_host_stage);
+  auto h2d = [&](size_t off, const void* src, size_t bytes) -> cudaError_t {
+    return bytes ? cudaMemcpyAsync(d + off, src, bytes, cudaMemcpyHostToDevice, stream) : cudaSuccess;
+  };
+  DSA_CUDA_TRY(h2d(0, k_new_host, b_k), "cudaMemcpyAsync(k_new)");
+  DSA_CUDA_TRY(h2d(o_rows, dst_rows_host, b_rows), "cudaMemcpyAsync(dst_rows)");
+  DSA_CUDA_TRY(h2d(o_q, q->data, b_q), "cudaMemcpyAsync(q)");
+  DSA_CUDA_TRY(h2d(o_qs, q->scale, b_qs), "cudaMemcpyAsync(q_scale)");
+  DSA_CUDA_TRY(h2d(o_w, w_host, b_w), "cudaMemcpyAsync(w)");
+  if (n_new > 0 &&
+      (st = dsa_indexer_kcache_append(kc, d, k_new_dtype, reinterpret_cast<const int64_t*>(d + o_rows), n_new,
+                                      stream_v)) != DSA_OK)
+    return st;
+  dsa_query_t qd = *q;
+  qd.data = d + o_q;
+  qd.scale = b_qs ? reinterpret_cast<const float*>(d + o_qs) : nullptr;
+  if (quantise_q && T > 0) {
+    if ((st = dsa_quantize_rows_fp8(d + o_q, DSA_BF16, T, q->H_I * q->d_I, reinterpret_cast<uint8_t*>(d + o_q8),
+                                    reinterpret_cast<float*>(d + o_q8s), stream_v)) != DSA_OK)
+      return st;
+    qd.data = d + o_q8;
+    qd.scale = reinterpret_cast<const float*>(d + o_q8s);
+    qd.dtype = DSA_FP8_E4M3;
+  }
+  int32_t* oi = reinterpret_cast<int32_t*>(d + o_oi);
+  float* os = reinterpret_cast<float*>(d + o_os);
+  if ((st = dsa_indexer_decode(&qd, kc, reinterpret_cast<const float*>(d + o_w), batch, top_k, oi, os, stream_v)) !=
+      DSA_OK)
+    return st;
+  if (b_out) {
+    DSA_CUDA_TRY(cudaMemcpyAsync(out_idx_host, oi, b_out, cudaMemcpyDeviceToHost, stream), "cudaMemcpyAsync(out_idx)");
+    DSA_CUDA_TRY(cudaMemcpyAsync(out_score_host, os, b_out, cudaMemcpyDeviceToHost, stream), "cudaMemcpyAsync(out_score)");
+  }
+  return DSA_OK;
 }
 
 dsa_status_t dsa_indexer_scores(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,

@@ -344,6 +344,58 @@ def test_full_ragged_decode_fp8_sampled_sequences():
     _check(up, idx, sc, rows)
 
 
+# ----------------------------------------------------------------------------- one-call host step
+
+def _sorted_rows(idx, sc):
+    out = []
+    for r in range(idx.shape[0]):
+        o = np.lexsort((idx[r], -sc[r]))
+        out.append((idx[r][o], sc[r][o]))
+    return out
+
+
+@pytest.mark.parametrize("name", ["bf16", "fp8"])
+def test_decode_host_step_equals_device_calls_two_calls_in_a_row(name):
+    base = W.decode() if name == "bf16" else W.decode8()
+    lens = [(6000, 2100, 300, 4097), (5000, 2049, 3333, 1)]
+    for call, L in enumerate(lens):
+        q_lens = (1, 2, 1, 1)
+        wl = W.scaled(base, seq_lens=L, q_lens=q_lens, seed=50 + call)
+        up = Uploaded(wl)
+        ref_i, ref_s = _run(up, decode=True)
+        # the step re-appends each sequence's newest q_len keys (same values: the cache is unchanged)
+        rows = np.concatenate([up.k_base[b] + np.arange(Lb - n, Lb) for b, (Lb, n) in enumerate(zip(L, q_lens))])
+        k_bits = np.concatenate(up.inp["k_bits"])[rows]
+        k_h = torch.from_numpy(np.ascontiguousarray(k_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+        q_h = torch.from_numpy(np.ascontiguousarray(up.inp["q_bits"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        w_h = torch.from_numpy(up.inp["w"]).pin_memory()
+        rows_h = torch.from_numpy(rows.astype(np.int64)).pin_memory()
+        oi_h = torch.full((wl.total_q, wl.top_k), 7, dtype=torch.int32).pin_memory()
+        os_h = torch.zeros((wl.total_q, wl.top_k), dtype=torch.float32).pin_memory()
+        s = torch.cuda.current_stream()
+        api.dsa_indexer_decode_host(q_h, w_h, k_h, rows_h, up.cache, L, q_lens, wl.top_k, oi_h, os_h,
+                                    k_base=up.k_base, stream=s)
+        api.dsa_check_device_errors(s)                       # synchronises the stream
+        for (gi, gs), (ri, rs) in zip(_sorted_rows(oi_h.numpy(), os_h.numpy()), _sorted_rows(ref_i, ref_s)):
+            assert np.array_equal(gi, ri)
+            np.testing.assert_array_equal(gs, rs)
+
+
+def test_decode_host_step_rejects_bad_arguments():
+    wl = W.scaled(W.decode(), seq_lens=(300,), q_lens=(1,))
+    up = Uploaded(wl)
+    q_h = torch.zeros(1, 64, 128, dtype=torch.bfloat16)
+    w_h = torch.zeros(1, 64, dtype=torch.float32)
+    oi_h = torch.zeros(1, 16, dtype=torch.int32)
+    os_h = torch.zeros(1, 16, dtype=torch.float32)
+    with pytest.raises(ValueError, match="host tensors"):
+        api.dsa_indexer_decode_host(q_h.cuda(), w_h, None, torch.zeros(0, dtype=torch.int64), up.cache, (300,), (1,),
+                                    16, oi_h, os_h)
+    with pytest.raises(RuntimeError, match="INVALID_ARG"):
+        api.dsa_indexer_decode_host(q_h, w_h, None, torch.zeros(0, dtype=torch.int64), up.cache, (300,), (1,),
+                                    0, oi_h, os_h)
+
+
 # ----------------------------------------------------------------------------- CUDA graphs
 
 def test_graph_capture_replay_equals_eager_and_unplanned_capture_is_refused():
