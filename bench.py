@@ -267,6 +267,47 @@ def profiled_traffic():
         return None
 
 
+def after_select_timings(api, hx, stream, dev, reps=10):
+    """Latent-row gather (bf16 c^KV, d_c = 512 per cached token, synthetic) at the step's
+    selection, and the in-place sort of the selection; CUDA events around each launch, a
+    256 MB L2 flush before each."""
+    import torch
+    wl = hx.wl
+    with torch.cuda.stream(stream):
+        latent = torch.empty(wl.total_k, 512, dtype=torch.bfloat16, device=dev)
+        latent.view(torch.int16).random_()
+        base = api.selection_row_base(hx.seq_lens, hx.q_lens, hx.k_base, device=dev)
+        out = torch.empty(wl.total_q, wl.top_k, 512, dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        idx0, sc0 = hx.out_idx.clone(), hx.out_score.clone()
+    res = {}
+    for name in ("gather", "sort"):
+        total = 0.0
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                i2, s2 = idx0.clone(), sc0.clone()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            if name == "gather":
+                api.dsa_gather_rows(latent, idx0, base, out=out, stream=stream)
+            else:
+                api.dsa_sort_selection(i2, s2, stream=stream)
+            e1.record(stream)
+            stream.synchronize()
+            total += e0.elapsed_time(e1)
+        res[name] = total / reps
+    api.dsa_check_device_errors(stream)
+    valid = int((idx0 >= 0).sum().item())
+    moved = valid * 1024 + idx0.numel() * (4 + 1024) + base.numel() * 8   # reads of rows + idx, all writes
+    pk = peaks()
+    gbs = moved / (res["gather"] * 1e-3) / 1e9
+    del latent, out, flush
+    return {"gather_latent": {"ms": res["gather"], "rows": int(idx0.numel()), "row_bytes": 1024,
+                              "bytes": moved, "achieved_gbs": gbs, "frac_of_hbm": gbs / pk["hbm"]},
+            "sort_selection": {"ms": res["sort"], "rows": int(idx0.shape[0]), "top_k": int(idx0.shape[1])}}
+
+
 class Harness:
     """Device state and one step of the hot path for a workload.
 
@@ -487,6 +528,10 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in (k_h, q_h, w_h)) + (rows_h.numel() * 8 if hx.decode else 0)
     d2h = sum(t.numel() * t.element_size() for t in (oi_h, os_h))
 
+    # the selection's consumers (outside the timed step): the latent-row gather the sparse
+    # attention makes and the sorted order, each launch timed alone after an L2 flush
+    after = after_select_timings(api, hx, stream, dev) if hx.decode else None
+
     # roofline of the dominant kernel (the logits kernel)
     pk = peaks()
     if hx.decode:
@@ -530,6 +575,8 @@ def run_ours(args):
             "gpu_launches": int(round(launches_per_step * K)),
             "clocks": clk,
         }
+        if after is not None:
+            line["after_select"] = after
         print(json.dumps(line), flush=True)
     del graph
     if world > 1:

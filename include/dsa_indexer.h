@@ -215,6 +215,37 @@ DSA_API dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const dsa_
                                                 const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx,
                                                 float* out_score, int32_t* fault, void* stream);
 
+/*
+ * After the selection (what its consumers do with it).
+ *
+ * dsa_gather_rows: the sparse attention's read of the latent cache at the selected
+ * positions (page "Study MLA Indexer", section 数学流, and its 两条 cache 区分 table:
+ * c^KV, d_c = 512 per token; "Lightning Indexer 详解" §1):
+ *     dst[r, j, :] = src[row_base[r] + idx[r, j], :]   for idx[r, j] >= 0,
+ *     dst[r, j, :] = 0                                  for idx[r, j] == -1,
+ * with rows of row_bytes bytes (any element type; a multiple of 16, at most 4096).
+ *   src       device [src_rows, row_bytes], 16-byte aligned (e.g. the latent cache)
+ *   idx       device int32 [rows, top_k] (a selection from prefill / decode)
+ *   row_base  device int64 [rows]: cache row of position 0 of each query row's sequence
+ *   dst       device [rows, top_k, row_bytes], 16-byte aligned
+ * A source row outside [0, src_rows) is zero-filled and recorded as a device fault
+ * (dsa_check_device_errors).
+ *
+ * dsa_selection_rows: out[r, j] = row_base[r] + idx[r, j] (int64), -1 where idx is -1 —
+ * global cache rows for consumers that gather from one packed cache by int64 index.
+ *
+ * dsa_sort_selection: sorts every row of a selection in place by score descending, then
+ * position ascending, padding (-1 / -inf) last — the order torch.topk returns
+ * (-0.0 counts as, and is returned as, +0.0).  top_k <= 4096 (else DSA_ERR_UNSUPPORTED).
+ *
+ * All three only enqueue on `stream`.
+ */
+DSA_API dsa_status_t dsa_gather_rows(const void* src, int64_t src_rows, int32_t row_bytes, const int32_t* idx,
+                                     const int64_t* row_base, int64_t rows, int32_t top_k, void* dst, void* stream);
+DSA_API dsa_status_t dsa_selection_rows(const int32_t* idx, const int64_t* row_base, int64_t rows, int32_t top_k,
+                                        int64_t* out, void* stream);
+DSA_API dsa_status_t dsa_sort_selection(int32_t* idx, float* score, int64_t rows, int32_t top_k, void* stream);
+
 /* Workspace bytes a call with this batch needs (scores plus scheduling tables). */
 DSA_API size_t dsa_indexer_workspace_bytes(const dsa_query_t* q, const dsa_batch_t* batch, int32_t top_k);
 

@@ -25,6 +25,9 @@ EXPORTED = (
     "dsa_indexer_decode",
     "dsa_indexer_decode_noalloc",
     "dsa_indexer_decode_host",
+    "dsa_gather_rows",
+    "dsa_selection_rows",
+    "dsa_sort_selection",
     "dsa_indexer_scores",
     "dsa_indexer_workspace_bytes",
     "dsa_set_workspace",
@@ -83,6 +86,12 @@ def load() -> ctypes.CDLL:
     lib.dsa_indexer_decode_noalloc.restype = st
     lib.dsa_indexer_decode_host.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V, V]
     lib.dsa_indexer_decode_host.restype = st
+    lib.dsa_gather_rows.argtypes = [V, I64, I32, V, V, I64, I32, V, V]
+    lib.dsa_gather_rows.restype = st
+    lib.dsa_selection_rows.argtypes = [V, V, I64, I32, V, V]
+    lib.dsa_selection_rows.restype = st
+    lib.dsa_sort_selection.argtypes = [V, V, I64, I32, V]
+    lib.dsa_sort_selection.restype = st
     lib.dsa_indexer_scores.argtypes = [P(Query), P(KCache), V, P(Batch), V, I64, V]
     lib.dsa_indexer_scores.restype = st
     lib.dsa_indexer_workspace_bytes.argtypes = [P(Query), P(Batch), I32]

@@ -197,6 +197,52 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
                                               _ptr(out_score_host), _stream(stream)))
 
 
+def selection_row_base(seq_lens, q_lens=None, k_base=None, device="cuda"):
+    """int64 [T_total] device tensor: the cache row of position 0 of each packed query row's
+    sequence (what dsa_gather_rows / dsa_selection_rows add to the selected positions).
+    k_base None: sequences packed back to back from row 0; q_lens None: prefill (q_len = seq_len)."""
+    seq = np.asarray(seq_lens, dtype=np.int64)
+    ql = seq if q_lens is None else np.asarray(q_lens, dtype=np.int64)
+    base = np.concatenate([[0], np.cumsum(seq)[:-1]]) if k_base is None else np.asarray(k_base, dtype=np.int64)
+    return torch.from_numpy(np.repeat(base, ql).astype(np.int64)).to(device)
+
+
+def dsa_gather_rows(src, idx, row_base, out=None, stream=None):
+    """Gather the selected rows: out[r, j] = src[row_base[r] + idx[r, j]] (zeros for -1).
+    src [rows, ...] any dtype, contiguous, rows of a multiple of 16 bytes; idx int32 [T, k];
+    row_base int64 [T] (device).  Returns [T, k, ...] with src's dtype."""
+    _require_cuda(src, idx, row_base, out)
+    if idx.dtype != torch.int32 or row_base.dtype != torch.int64:
+        raise TypeError("idx must be int32 and row_base int64")
+    if not (src.is_contiguous() and idx.is_contiguous() and row_base.is_contiguous()):
+        raise ValueError("src, idx and row_base must be contiguous")
+    T, k = idx.shape
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else 0
+    if out is None:
+        out = torch.empty((T, k) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    check(_lib.load().dsa_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(idx), _ptr(row_base), T, k, _ptr(out),
+                                      _stream(stream)))
+    return out
+
+
+def dsa_selection_rows(idx, row_base, out=None, stream=None):
+    """int64 [T, k] cache rows of a selection: row_base[r] + idx[r, j], -1 where idx is -1."""
+    _require_cuda(idx, row_base, out)
+    T, k = idx.shape
+    if out is None:
+        out = torch.empty(T, k, dtype=torch.int64, device=idx.device)
+    check(_lib.load().dsa_selection_rows(_ptr(idx), _ptr(row_base), T, k, _ptr(out), _stream(stream)))
+    return out
+
+
+def dsa_sort_selection(idx, score, stream=None):
+    """Sort each row of a selection in place: score descending, then position ascending, padding last."""
+    _require_cuda(idx, score)
+    T, k = idx.shape
+    check(_lib.load().dsa_sort_selection(_ptr(idx), _ptr(score), T, k, _stream(stream)))
+    return idx, score
+
+
 def dsa_indexer_scores(q, cache: IndexerKCache, w, seq_lens, q_scale=None, q_lens=None, k_base=None, ld=None,
                        out=None, stream=None):
     """Dense scores [T_total, ld] (entries after each query's position are left as they were: -inf here)."""

@@ -888,6 +888,59 @@ dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* k
   return DSA_OK;
 }
 
+dsa_status_t dsa_gather_rows(const void* src, int64_t src_rows, int32_t row_bytes, const int32_t* idx,
+                             const int64_t* row_base, int64_t rows, int32_t top_k, void* dst, void* stream_v) {
+  g_last_error.clear();
+  if (rows < 0 || top_k < 0 || src_rows < 0) return fail(DSA_ERR_INVALID_ARG, "negative size");
+  if (rows == 0 || top_k == 0) return DSA_OK;
+  if (!src || !idx || !row_base || !dst) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!gather_row_bytes_supported(row_bytes))
+    return fail(DSA_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16, at most 4096");
+  if (reinterpret_cast<uintptr_t>(src) % 16 || reinterpret_cast<uintptr_t>(dst) % 16)
+    return fail(DSA_ERR_INVALID_ARG, "src and dst must be 16-byte aligned");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  Ctx* c = nullptr;
+  dsa_status_t st = get_ctx(stream, &c);
+  if (st != DSA_OK) return st;
+  if (!g_sms) g_sms = num_sms(c->device);
+  DSA_CUDA_TRY(launch_gather_rows(src, src_rows, row_bytes, idx, row_base, rows, top_k, dst, c->d_err, g_sms, stream),
+               "gather kernel launch");
+  ++g_launches;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_selection_rows(const int32_t* idx, const int64_t* row_base, int64_t rows, int32_t top_k,
+                                int64_t* out, void* stream_v) {
+  g_last_error.clear();
+  if (rows < 0 || top_k < 0) return fail(DSA_ERR_INVALID_ARG, "negative size");
+  if (rows == 0 || top_k == 0) return DSA_OK;
+  if (!idx || !row_base || !out) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  Ctx* c = nullptr;
+  dsa_status_t st = get_ctx(stream, &c);
+  if (st != DSA_OK) return st;
+  if (!g_sms) g_sms = num_sms(c->device);
+  DSA_CUDA_TRY(launch_selection_rows(idx, row_base, rows, top_k, out, g_sms, stream), "selection-rows kernel launch");
+  ++g_launches;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_sort_selection(int32_t* idx, float* score, int64_t rows, int32_t top_k, void* stream_v) {
+  g_last_error.clear();
+  if (rows < 0 || top_k < 0) return fail(DSA_ERR_INVALID_ARG, "negative size");
+  if (rows == 0 || top_k <= 1) return DSA_OK;
+  if (!idx || !score) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (top_k > sort_selection_max()) return fail(DSA_ERR_UNSUPPORTED, "dsa_sort_selection takes top_k <= %d", sort_selection_max());
+  if (rows > 0x7FFFFFFF) return fail(DSA_ERR_UNSUPPORTED, "too many rows for one launch");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  Ctx* c = nullptr;
+  dsa_status_t st = get_ctx(stream, &c);
+  if (st != DSA_OK) return st;
+  DSA_CUDA_TRY(launch_sort_selection(idx, score, rows, top_k, stream), "sort kernel launch");
+  ++g_launches;
+  return DSA_OK;
+}
+
 dsa_status_t dsa_indexer_scores(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
                                 const dsa_batch_t* batch, float* out_scores, int64_t ld, void* stream) {
   return run_indexer(Mode::Scores, q, kc, w, batch, 1, nullptr, nullptr, out_scores, ld, stream);

@@ -114,6 +114,16 @@ cudaError_t launch_topk_stream(const TopkArgs& a, cudaStream_t stream);
 // Rows with at most top_k candidates: every causal position, then padding.
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream);
 
+// After the selection: latent-row gather, int64 cache rows, sorted order.
+bool gather_row_bytes_supported(int32_t row_bytes);
+int sort_selection_max();
+cudaError_t launch_gather_rows(const void* src, int64_t src_rows, int32_t row_bytes, const int32_t* idx,
+                               const int64_t* row_base, int64_t rows, int32_t top_k, void* dst, int* err, int sms,
+                               cudaStream_t stream);
+cudaError_t launch_selection_rows(const int32_t* idx, const int64_t* row_base, int64_t rows, int32_t top_k,
+                                  int64_t* out, int sms, cudaStream_t stream);
+cudaError_t launch_sort_selection(int32_t* idx, float* score, int64_t rows, int32_t top_k, cudaStream_t stream);
+
 cudaError_t launch_quantize_rows_fp8(const void* src, int src_is_f32, int64_t rows, int32_t row_len,
                                      uint8_t* dst, float* scale, const int64_t* dst_rows, int64_t dst_capacity,
                                      int* err, cudaStream_t stream);

@@ -1,0 +1,182 @@
+// What the consumers of a selection do with it.
+//
+// * Gather of the selected latent rows: the sparse MQA after the indexer reads the latent
+//   c^KV only at the top-k positions (page "Study MLA Indexer", section 数学流; its 两条
+//   cache 区分 table: d_c = 512 values per token; "Lightning Indexer 详解" §1: Core MLA
+//   attends only over the index set).  dst[r, j, :] = src[row_base[r] + idx[r, j], :],
+//   zero rows for -1.  Rows are opaque bytes (any dtype), moved as 16-byte vectors, one
+//   warp per output row.  HBM-bound: row_bytes read + row_bytes written per entry.
+// * Global cache rows of a selection, int64 (for consumers indexing one packed cache).
+// * Sorted selection: each row by score descending, then position ascending, padding last
+//   (the order torch.topk returns, the first page §3 step 5).  One CTA per row sorts
+//   64-bit composite keys (order key of the score, complemented position) in shared memory
+//   with a bitonic network.
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kGatherThreads = 256;
+constexpr int kMaxRowVecs = 32 * 8;           // rows up to 4 KB: at most 8 vectors per lane
+
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4* __restrict__ src, int64_t src_rows,
+                                                                     int32_t row_vecs, const int32_t* __restrict__ idx,
+                                                                     const int64_t* __restrict__ row_base,
+                                                                     int64_t n_out, int32_t top_k,
+                                                                     uint4* __restrict__ dst, int* err) {
+  grid_dependency_wait();                     // the selection comes from the previous kernel
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kGatherThreads + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kGatherThreads) >> 5;
+  for (int64_t o = warp0; o < n_out; o += n_warps) {
+    const int64_t r = o / top_k;
+    const int32_t i = idx[o];
+    int64_t srow = -1;
+    if (i >= 0) {
+      srow = row_base[r] + i;
+      if (srow < 0 || srow >= src_rows) {
+        if (lane == 0) record_error(err, DSA_DEVERR_BOUNDS, static_cast<int>(r));
+        srow = -1;
+      }
+    }
+    uint4* d = dst + o * row_vecs;
+    if (srow >= 0) {
+      const uint4* s = src + srow * row_vecs;
+      uint4 v[kMaxRowVecs / 32];
+#pragma unroll
+      for (int u = 0; u < kMaxRowVecs / 32; ++u) {       // every load of the row in flight together
+        const int c = u * 32 + lane;
+        if (c < row_vecs) v[u] = __ldcs(s + c);
+      }
+#pragma unroll
+      for (int u = 0; u < kMaxRowVecs / 32; ++u) {
+        const int c = u * 32 + lane;
+        if (c < row_vecs) __stcs(d + c, v[u]);
+      }
+    } else {
+      for (int c = lane; c < row_vecs; c += 32) d[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) selection_rows_kernel(const int32_t* __restrict__ idx,
+                                                             const int64_t* __restrict__ row_base, int64_t n_out,
+                                                             int32_t top_k, int64_t* __restrict__ out) {
+  grid_dependency_wait();
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < n_out;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int32_t i = idx[o];
+    out[o] = i >= 0 ? row_base[o / top_k] + i : -1;
+  }
+}
+
+constexpr int kSortThreads = 512;
+constexpr int kSortMax = 4096;                // entries per row the shared-memory sort takes
+
+__global__ void __launch_bounds__(kSortThreads) sort_selection_kernel(int32_t* __restrict__ idx,
+                                                                      float* __restrict__ score, int32_t top_k,
+                                                                      int32_t width) {
+  __shared__ unsigned long long key[kSortMax];
+  grid_dependency_wait();
+  int32_t* oi = idx + static_cast<int64_t>(blockIdx.x) * top_k;
+  float* os = score + static_cast<int64_t>(blockIdx.x) * top_k;
+  const int tid = threadIdx.x;
+  // key: order key of the score (high word), ~position (low word); padding 0 sorts last
+  for (int i = tid; i < width; i += kSortThreads) {
+    unsigned long long kk = 0ull;
+    if (i < top_k) {
+      const int32_t p = oi[i];
+      if (p >= 0)                             // + 0.0f: -0.0 ties with +0.0 (returned as +0.0)
+        kk = (static_cast<unsigned long long>(order_key(__float_as_uint(os[i] + 0.0f))) << 32) |
+             static_cast<unsigned long long>(~static_cast<uint32_t>(p));
+    }
+    key[i] = kk;
+  }
+  __syncthreads();
+  // bitonic network, descending overall
+  for (int size = 2; size <= width; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = tid; t < width / 2; t += kSortThreads) {
+        const int pos = 2 * t - (t & (stride - 1));
+        const int partner = pos + stride;
+        const bool desc = (pos & size) == 0;
+        const unsigned long long a = key[pos], b = key[partner];
+        if ((a < b) == desc) {
+          key[pos] = b;
+          key[partner] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < top_k; i += kSortThreads) {
+    const unsigned long long kk = key[i];
+    if (kk == 0ull) {
+      oi[i] = -1;
+      os[i] = -INFINITY;
+    } else {
+      oi[i] = static_cast<int32_t>(~static_cast<uint32_t>(kk & 0xFFFFFFFFull));
+      const uint32_t u = static_cast<uint32_t>(kk >> 32);
+      os[i] = __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+    }
+  }
+}
+
+cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t stream, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+}  // namespace
+
+bool gather_row_bytes_supported(int32_t row_bytes) {
+  return row_bytes > 0 && row_bytes % 16 == 0 && row_bytes / 16 <= kMaxRowVecs;
+}
+
+int sort_selection_max() { return kSortMax; }
+
+cudaError_t launch_gather_rows(const void* src, int64_t src_rows, int32_t row_bytes, const int32_t* idx,
+                               const int64_t* row_base, int64_t rows, int32_t top_k, void* dst, int* err, int sms,
+                               cudaStream_t stream) {
+  const int64_t n_out = rows * top_k;
+  if (n_out == 0) return cudaSuccess;
+  const int64_t want = (n_out + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
+  const int64_t cap = static_cast<int64_t>(sms) * (2048 / kGatherThreads) * 4;   // a few waves' worth
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(want < cap ? want : cap)), dim3(kGatherThreads),
+                                      stream, attr);
+  return cudaLaunchKernelEx(&cfg, gather_rows_kernel, static_cast<const uint4*>(src), src_rows, row_bytes / 16, idx,
+                            row_base, n_out, top_k, static_cast<uint4*>(dst), err);
+}
+
+cudaError_t launch_selection_rows(const int32_t* idx, const int64_t* row_base, int64_t rows, int32_t top_k,
+                                  int64_t* out, int sms, cudaStream_t stream) {
+  const int64_t n_out = rows * top_k;
+  if (n_out == 0) return cudaSuccess;
+  const int64_t want = (n_out + 255) / 256, cap = static_cast<int64_t>(sms) * 8;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(want < cap ? want : cap)), dim3(256), stream, attr);
+  return cudaLaunchKernelEx(&cfg, selection_rows_kernel, idx, row_base, n_out, top_k, out);
+}
+
+cudaError_t launch_sort_selection(int32_t* idx, float* score, int64_t rows, int32_t top_k, cudaStream_t stream) {
+  if (rows == 0 || top_k <= 1) return cudaSuccess;
+  int32_t width = 2;
+  while (width < top_k) width <<= 1;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(rows)), dim3(kSortThreads), stream, attr);
+  return cudaLaunchKernelEx(&cfg, sort_selection_kernel, idx, score, top_k, width);
+}
+
+}  // namespace dsa
