@@ -269,8 +269,9 @@ def profiled_traffic():
 
 def after_select_timings(api, hx, stream, dev, reps=10):
     """Latent-row gather (bf16 c^KV, d_c = 512 per cached token, synthetic) at the step's
-    selection, and the in-place sort of the selection; CUDA events around each launch, a
-    256 MB L2 flush before each."""
+    selection, and the in-place sort of the selection; CUDA events around each launch.  Before
+    each launch a 256 MB buffer is read (not written): that evicts the inputs from the L2
+    without leaving dirty lines whose write-back would fall into the timed launch."""
     import torch
     wl = hx.wl
     with torch.cuda.stream(stream):
@@ -278,14 +279,14 @@ def after_select_timings(api, hx, stream, dev, reps=10):
         latent.view(torch.int16).random_()
         base = api.selection_row_base(hx.seq_lens, hx.q_lens, hx.k_base, device=dev)
         out = torch.empty(wl.total_q, wl.top_k, 512, dtype=torch.bfloat16, device=dev)
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
         idx0, sc0 = hx.out_idx.clone(), hx.out_score.clone()
     res = {}
     for name in ("gather", "sort"):
         total = 0.0
         for _ in range(reps):
             with torch.cuda.stream(stream):
-                flush.zero_()
+                flush.max()
                 i2, s2 = idx0.clone(), sc0.clone()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)

@@ -22,44 +22,56 @@ namespace {
 
 constexpr int kGatherThreads = 256;
 constexpr int kMaxRowVecs = 32 * 8;           // rows up to 4 KB: at most 8 vectors per lane
+constexpr int kGatherInFlight = 8;            // 16-byte loads per lane issued together
 
+// One warp copies RPW rows per iteration, VPL vectors per lane per row (VPL * 32 >= the
+// row's vectors), all RPW * VPL loads of the iteration in flight before any store.
+template <int VPL, int RPW>
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4* __restrict__ src, int64_t src_rows,
                                                                      int32_t row_vecs, const int32_t* __restrict__ idx,
                                                                      const int64_t* __restrict__ row_base,
                                                                      int64_t n_out, int32_t top_k,
                                                                      uint4* __restrict__ dst, int* err) {
+  static_assert(VPL * RPW == kGatherInFlight, "loads in flight per lane");
   grid_dependency_wait();                     // the selection comes from the previous kernel
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kGatherThreads + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kGatherThreads) >> 5;
-  for (int64_t o = warp0; o < n_out; o += n_warps) {
-    const int64_t r = o / top_k;
-    const int32_t i = idx[o];
-    int64_t srow = -1;
-    if (i >= 0) {
-      srow = row_base[r] + i;
-      if (srow < 0 || srow >= src_rows) {
-        if (lane == 0) record_error(err, DSA_DEVERR_BOUNDS, static_cast<int>(r));
-        srow = -1;
+  for (int64_t o0 = warp0 * RPW; o0 < n_out; o0 += n_warps * RPW) {
+    int64_t srow[RPW];
+#pragma unroll
+    for (int q = 0; q < RPW; ++q) {
+      const int64_t o = o0 + q;
+      srow[q] = -2;                                       // -2: no such output row
+      if (o < n_out) {
+        const int32_t i = idx[o];
+        srow[q] = -1;
+        if (i >= 0) {
+          const int64_t sr = row_base[o / top_k] + i;
+          if (sr < 0 || sr >= src_rows) {
+            if (lane == 0) record_error(err, DSA_DEVERR_BOUNDS, static_cast<int>(o / top_k));
+          } else {
+            srow[q] = sr;
+          }
+        }
       }
     }
-    uint4* d = dst + o * row_vecs;
-    if (srow >= 0) {
-      const uint4* s = src + srow * row_vecs;
-      uint4 v[kMaxRowVecs / 32];
+    uint4 v[RPW][VPL];
 #pragma unroll
-      for (int u = 0; u < kMaxRowVecs / 32; ++u) {       // every load of the row in flight together
+    for (int q = 0; q < RPW; ++q)
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
         const int c = u * 32 + lane;
-        if (c < row_vecs) v[u] = __ldcs(s + c);
+        v[q][u] = make_uint4(0u, 0u, 0u, 0u);
+        if (srow[q] >= 0 && c < row_vecs) v[q][u] = __ldcs(src + srow[q] * row_vecs + c);
       }
 #pragma unroll
-      for (int u = 0; u < kMaxRowVecs / 32; ++u) {
+    for (int q = 0; q < RPW; ++q)
+#pragma unroll
+      for (int u = 0; u < VPL; ++u) {
         const int c = u * 32 + lane;
-        if (c < row_vecs) __stcs(d + c, v[u]);
+        if (srow[q] != -2 && c < row_vecs) __stcs(dst + (o0 + q) * row_vecs + c, v[q][u]);
       }
-    } else {
-      for (int c = lane; c < row_vecs; c += 32) d[c] = make_uint4(0u, 0u, 0u, 0u);
-    }
   }
 }
 
@@ -97,7 +109,9 @@ __global__ void __launch_bounds__(kSortThreads) sort_selection_kernel(int32_t* _
     key[i] = kk;
   }
   __syncthreads();
-  // bitonic network, descending overall
+  // bitonic network, descending overall.  A stage of stride <= 16 touches, for each t, only
+  // the 64-element block of its warp's t range, so only a stage of stride >= 32 (or the end)
+  // needs the whole CTA to have finished the stage before it.
   for (int size = 2; size <= width; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       for (int t = tid; t < width / 2; t += kSortThreads) {
@@ -110,7 +124,11 @@ __global__ void __launch_bounds__(kSortThreads) sort_selection_kernel(int32_t* _
           key[partner] = a;
         }
       }
-      __syncthreads();
+      const int next_stride = stride > 1 ? stride >> 1 : size;   // the next stage's stride
+      if (next_stride >= 32 || (stride == 1 && size == width))
+        __syncthreads();
+      else
+        __syncwarp();
     }
   }
   for (int i = tid; i < top_k; i += kSortThreads) {
@@ -151,13 +169,22 @@ cudaError_t launch_gather_rows(const void* src, int64_t src_rows, int32_t row_by
                                cudaStream_t stream) {
   const int64_t n_out = rows * top_k;
   if (n_out == 0) return cudaSuccess;
-  const int64_t want = (n_out + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
-  const int64_t cap = static_cast<int64_t>(sms) * (2048 / kGatherThreads) * 4;   // a few waves' worth
+  const int32_t row_vecs = row_bytes / 16;
+  const int vpl = row_vecs <= 32 ? 1 : row_vecs <= 64 ? 2 : row_vecs <= 128 ? 4 : 8;
+  const int rpw = kGatherInFlight / vpl;
+  const int64_t want = (n_out + rpw * (kGatherThreads / 32) - 1) / (rpw * (kGatherThreads / 32));
+  const int64_t cap = static_cast<int64_t>(sms) * 4;     // one resident wave (about 64 registers a thread)
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(want < cap ? want : cap)), dim3(kGatherThreads),
                                       stream, attr);
-  return cudaLaunchKernelEx(&cfg, gather_rows_kernel, static_cast<const uint4*>(src), src_rows, row_bytes / 16, idx,
-                            row_base, n_out, top_k, static_cast<uint4*>(dst), err);
+  const uint4* s = static_cast<const uint4*>(src);
+  uint4* d = static_cast<uint4*>(dst);
+  switch (vpl) {
+    case 1: return cudaLaunchKernelEx(&cfg, gather_rows_kernel<1, 8>, s, src_rows, row_vecs, idx, row_base, n_out, top_k, d, err);
+    case 2: return cudaLaunchKernelEx(&cfg, gather_rows_kernel<2, 4>, s, src_rows, row_vecs, idx, row_base, n_out, top_k, d, err);
+    case 4: return cudaLaunchKernelEx(&cfg, gather_rows_kernel<4, 2>, s, src_rows, row_vecs, idx, row_base, n_out, top_k, d, err);
+    default: return cudaLaunchKernelEx(&cfg, gather_rows_kernel<8, 1>, s, src_rows, row_vecs, idx, row_base, n_out, top_k, d, err);
+  }
 }
 
 cudaError_t launch_selection_rows(const int32_t* idx, const int64_t* row_base, int64_t rows, int32_t top_k,
