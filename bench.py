@@ -309,6 +309,52 @@ def after_select_timings(api, hx, stream, dev, reps=10):
             "sort_selection": {"ms": res["sort"], "rows": int(idx0.shape[0]), "top_k": int(idx0.shape[1])}}
 
 
+def rope_timings(api, stream, dev, reps=10):
+    """The fused RoPE kernels at prefill size (16384 tokens, H_I = 64, d_I = 128): queries
+    rotated and quantised to E4M3, and 65536 key rows rotated and quantised into an FP8 cache;
+    CUDA events around each launch after a 256 MB L2-evicting read."""
+    import torch
+    T, H, d, n = 16384, 64, 128, 65536
+    with torch.cuda.stream(stream):
+        q = torch.randn(T, H, d, device=dev).to(torch.bfloat16)
+        pos_q = torch.arange(T, dtype=torch.int32, device=dev)
+        k = torch.randn(n, d, device=dev).to(torch.bfloat16)
+        pos_k = torch.arange(n, dtype=torch.int32, device=dev)
+        rows = torch.arange(n, dtype=torch.int64, device=dev)
+        cache = api.IndexerKCache.empty(n, d, True, device=dev)
+        codes = torch.empty(T, H, d, dtype=torch.uint8, device=dev)
+        scale = torch.empty(T, dtype=torch.float32, device=dev)
+        flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    res = {}
+    for name in ("queries", "keys"):
+        total = 0.0
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                flush.max()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            if name == "queries":
+                api.dsa_rope_queries(q, pos_q, fp8=True, rope_dim=64, interleaved=False, out=codes, scale=scale,
+                                     stream=stream)
+            else:
+                api.dsa_indexer_kcache_append_rope(cache, k, rows, pos_k, rope_dim=64, interleaved=False, stream=stream)
+            e1.record(stream)
+            stream.synchronize()
+            total += e0.elapsed_time(e1)
+        res[name] = total / reps
+    api.dsa_check_device_errors(stream)
+    hbm = peaks()["hbm"]
+    qb = T * H * d * 2 + T * 4 + T * H * d + T * 4          # bf16 in, positions, codes + scales out
+    kb = n * d * 2 + n * 12 + n * d + n * 4                 # bf16 in, positions + rows, codes + scales out
+    out = {}
+    for name, b in (("queries", qb), ("keys", kb)):
+        gbs = b / (res[name] * 1e-3) / 1e9
+        out[name] = {"ms": res[name], "bytes": b, "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm}
+    out["config"] = "16384 queries x 64 heads / 65536 keys, d_I=128, rope_dim 64 (half pairs), FP8 out"
+    del q, k, cache, codes, flush
+    return out
+
+
 class Harness:
     """Device state and one step of the hot path for a workload.
 
@@ -532,6 +578,7 @@ def run_ours(args):
     # the selection's consumers (outside the timed step): the latent-row gather the sparse
     # attention makes and the sorted order, each launch timed alone after an L2 flush
     after = after_select_timings(api, hx, stream, dev) if hx.decode else None
+    rope = rope_timings(api, stream, dev) if hx.decode else None
 
     # roofline of the dominant kernel (the logits kernel)
     pk = peaks()
@@ -578,6 +625,8 @@ def run_ours(args):
         }
         if after is not None:
             line["after_select"] = after
+        if rope is not None:
+            line["rope_fused"] = rope
         print(json.dumps(line), flush=True)
     del graph
     if world > 1:

@@ -216,6 +216,40 @@ DSA_API dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const dsa_
                                                 float* out_score, int32_t* fault, void* stream);
 
 /*
+ * Rotary position embedding of indexer keys and queries, fused into the cache append and
+ * the query quantisation (page "Study MLA Indexer", section 数学流: the key is RoPE'd, then
+ * quantised and written to the indexer K cache; the query is RoPE'd).  The pages give no
+ * RoPE detail; this is the published rotary embedding: pair i of the first rope_dim values
+ * of each d_I-vector turns by theta_i = position * base^(-2i / rope_dim),
+ * (a, b) -> (a cos - b sin, a sin + b cos); later values pass through.
+ */
+typedef struct {
+  int32_t rope_dim;     /* leading values that rotate: even, <= d_I (0: none)               */
+  int32_t interleaved;  /* 1: pairs (2i, 2i+1); 0: pairs (i, i + rope_dim/2), which needs     */
+                        /*    rope_dim / 2 = 2^m * d_I / 32 (e.g. d_I = 128: 8, 16, 32, 64, 128)   */
+  double base;          /* 10000 in the published form                                        */
+} dsa_rope_t;
+
+/*
+ * dsa_indexer_kcache_append with the rotation first: key row r (k_new [n, d_I], bf16 or
+ * fp32, pre-RoPE) is rotated at position positions[r] (device int32 [n]) and stored at cache
+ * row dst_rows[r] as bf16 or quantised E4M3 + scale, like dsa_indexer_kcache_append.
+ */
+DSA_API dsa_status_t dsa_indexer_kcache_append_rope(const dsa_kcache_t* kc, const void* k_new, dsa_dtype_t src_dtype,
+                                                    const int64_t* dst_rows, const int32_t* positions, int32_t n,
+                                                    const dsa_rope_t* rope, void* stream);
+
+/*
+ * Queries q_src [T, H_I, d_I] (bf16 or fp32, pre-RoPE, device): every head of token t is
+ * rotated at positions[t] (device int32 [T]) and written to q_dst [T, H_I, d_I] as bf16
+ * (dst_dtype DSA_BF16) or as E4M3 codes with one scale per token in q_scale [T]
+ * (DSA_FP8_E4M3, as dsa_quantize_rows_fp8).  H_I <= 128, d_I 64 or 128.
+ */
+DSA_API dsa_status_t dsa_rope_queries(const void* q_src, dsa_dtype_t src_dtype, int64_t T, int32_t H_I, int32_t d_I,
+                                      const int32_t* positions, const dsa_rope_t* rope, void* q_dst,
+                                      dsa_dtype_t dst_dtype, float* q_scale, void* stream);
+
+/*
  * After the selection (what its consumers do with it).
  *
  * dsa_gather_rows: the sparse attention's read of the latent cache at the selected

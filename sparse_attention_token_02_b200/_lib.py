@@ -25,6 +25,8 @@ EXPORTED = (
     "dsa_indexer_decode",
     "dsa_indexer_decode_noalloc",
     "dsa_indexer_decode_host",
+    "dsa_indexer_kcache_append_rope",
+    "dsa_rope_queries",
     "dsa_gather_rows",
     "dsa_selection_rows",
     "dsa_sort_selection",
@@ -42,6 +44,10 @@ EXPORTED = (
 class KCache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("capacity_rows", ctypes.c_int64),
                 ("d_I", ctypes.c_int32), ("dtype", ctypes.c_int)]
+
+
+class Rope(ctypes.Structure):
+    _fields_ = [("rope_dim", ctypes.c_int32), ("interleaved", ctypes.c_int32), ("base", ctypes.c_double)]
 
 
 class Query(ctypes.Structure):
@@ -86,6 +92,10 @@ def load() -> ctypes.CDLL:
     lib.dsa_indexer_decode_noalloc.restype = st
     lib.dsa_indexer_decode_host.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V, V]
     lib.dsa_indexer_decode_host.restype = st
+    lib.dsa_indexer_kcache_append_rope.argtypes = [P(KCache), V, ctypes.c_int, V, V, I32, P(Rope), V]
+    lib.dsa_indexer_kcache_append_rope.restype = st
+    lib.dsa_rope_queries.argtypes = [V, ctypes.c_int, I64, I32, I32, V, P(Rope), V, ctypes.c_int, V, V]
+    lib.dsa_rope_queries.restype = st
     lib.dsa_gather_rows.argtypes = [V, I64, I32, V, V, I64, I32, V, V]
     lib.dsa_gather_rows.restype = st
     lib.dsa_selection_rows.argtypes = [V, V, I64, I32, V, V]

@@ -197,6 +197,45 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
                                               _ptr(out_score_host), _stream(stream)))
 
 
+def _rope(d, rope_dim, base, interleaved):
+    from ._lib import Rope
+    return Rope(d if rope_dim is None else int(rope_dim), 1 if interleaved else 0, float(base))
+
+
+def dsa_indexer_kcache_append_rope(cache: IndexerKCache, k_new, dst_rows, positions, rope_dim=None, base=10000.0,
+                                   interleaved=True, stream=None):
+    """Rotate pre-RoPE key rows k_new [n, d_I] (bf16/fp32) at ``positions`` (int32 [n]) and append
+    them at cache rows ``dst_rows`` (int64 [n]); FP8 caches get the quantised rows + scales.
+    rope_dim None rotates the whole vector."""
+    _require_cuda(k_new, dst_rows, positions)
+    if dst_rows.dtype != torch.int64 or positions.dtype != torch.int32:
+        raise TypeError("dst_rows must be int64 and positions int32")
+    r = _rope(cache.k.shape[1], rope_dim, base, interleaved)
+    kc = cache.c()
+    check(_lib.load().dsa_indexer_kcache_append_rope(ctypes.byref(kc), _ptr(k_new.contiguous()), _dtype_code(k_new),
+                                                     _ptr(dst_rows), _ptr(positions), int(k_new.shape[0]),
+                                                     ctypes.byref(r), _stream(stream)))
+
+
+def dsa_rope_queries(q_src, positions, fp8=False, rope_dim=None, base=10000.0, interleaved=True, out=None,
+                     scale=None, stream=None):
+    """Rotate pre-RoPE queries q_src [T, H, d] (bf16/fp32) at ``positions`` (int32 [T]); returns
+    bf16 [T, H, d], or (uint8 E4M3 codes [T, H, d], fp32 scale [T]) with fp8=True."""
+    _require_cuda(q_src, positions, out, scale)
+    if positions.dtype != torch.int32:
+        raise TypeError("positions must be int32")
+    T, H, d = q_src.shape
+    if out is None:
+        out = torch.empty(T, H, d, dtype=torch.uint8 if fp8 else torch.bfloat16, device=q_src.device)
+    if fp8 and scale is None:
+        scale = torch.empty(T, dtype=torch.float32, device=q_src.device)
+    r = _rope(d, rope_dim, base, interleaved)
+    src = q_src.contiguous()
+    check(_lib.load().dsa_rope_queries(_ptr(src), _dtype_code(src), T, H, d, _ptr(positions), ctypes.byref(r),
+                                       _ptr(out), DSA_FP8_E4M3 if fp8 else DSA_BF16, _ptr(scale), _stream(stream)))
+    return (out, scale) if fp8 else out
+
+
 def selection_row_base(seq_lens, q_lens=None, k_base=None, device="cuda"):
     """int64 [T_total] device tensor: the cache row of position 0 of each packed query row's
     sequence (what dsa_gather_rows / dsa_selection_rows add to the selected positions).

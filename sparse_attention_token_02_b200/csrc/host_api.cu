@@ -730,6 +730,17 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
 
 }  // namespace
 
+// RoPE parameters for the kernels, with the pair frequencies base^(-2i / rope_dim) in fp64
+RopeParams rope_params(const dsa_rope_t& r) {
+  RopeParams p{};
+  p.rope_dim = r.rope_dim;
+  p.interleaved = r.interleaved;
+  p.base = r.base;
+  for (int i = 0; i < kRopeMaxPairs; ++i)
+    p.inv_freq[i] = (r.rope_dim > 0 && r.base > 0.0) ? std::pow(r.base, -2.0 * i / r.rope_dim) : 0.0;
+  return p;
+}
+
 int num_sms(int device) {
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) n = 148;
@@ -885,6 +896,53 @@ dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* k
     DSA_CUDA_TRY(cudaMemcpyAsync(out_idx_host, oi, b_out, cudaMemcpyDeviceToHost, stream), "cudaMemcpyAsync(out_idx)");
     DSA_CUDA_TRY(cudaMemcpyAsync(out_score_host, os, b_out, cudaMemcpyDeviceToHost, stream), "cudaMemcpyAsync(out_score)");
   }
+  return DSA_OK;
+}
+
+dsa_status_t dsa_indexer_kcache_append_rope(const dsa_kcache_t* kc, const void* k_new, dsa_dtype_t src_dtype,
+                                            const int64_t* dst_rows, const int32_t* positions, int32_t n,
+                                            const dsa_rope_t* rope, void* stream_v) {
+  g_last_error.clear();
+  dsa_status_t st = check_cache(kc);
+  if (st != DSA_OK) return st;
+  if (n < 0) return fail(DSA_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return DSA_OK;
+  if (!k_new || !dst_rows || !positions || !rope) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (src_dtype != DSA_BF16 && src_dtype != DSA_F32) return fail(DSA_ERR_INVALID_ARG, "src_dtype must be DSA_BF16 or DSA_F32");
+  const RopeParams rp = rope_params(*rope);
+  if (!rope_shape_supported(kc->d_I, 1, rp)) return fail(DSA_ERR_UNSUPPORTED, "unsupported RoPE layout for d_I = %d", kc->d_I);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  Ctx* c = nullptr;
+  if ((st = get_ctx(stream, &c)) != DSA_OK) return st;
+  const int fp8 = kc->dtype == DSA_FP8_E4M3;
+  DSA_CUDA_TRY(launch_rope_append(k_new, src_dtype == DSA_F32, n, kc->d_I, dst_rows, positions, kc->capacity_rows, rp,
+                                  fp8, kc->k, kc->k_scale, c->d_err, stream),
+               "RoPE append kernel launch");
+  ++g_launches;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_rope_queries(const void* q_src, dsa_dtype_t src_dtype, int64_t T, int32_t H, int32_t d,
+                              const int32_t* positions, const dsa_rope_t* rope, void* q_dst, dsa_dtype_t dst_dtype,
+                              float* q_scale, void* stream_v) {
+  g_last_error.clear();
+  if (T < 0) return fail(DSA_ERR_INVALID_ARG, "T < 0");
+  if (T == 0) return DSA_OK;
+  if (!q_src || !positions || !rope || !q_dst) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (src_dtype != DSA_BF16 && src_dtype != DSA_F32) return fail(DSA_ERR_INVALID_ARG, "src_dtype must be DSA_BF16 or DSA_F32");
+  if (dst_dtype != DSA_BF16 && dst_dtype != DSA_FP8_E4M3) return fail(DSA_ERR_INVALID_ARG, "dst_dtype must be DSA_BF16 or DSA_FP8_E4M3");
+  if (dst_dtype == DSA_FP8_E4M3 && !q_scale) return fail(DSA_ERR_INVALID_ARG, "FP8 output needs q_scale");
+  if (T > 0x7FFFFFFF) return fail(DSA_ERR_UNSUPPORTED, "too many tokens for one launch");
+  const RopeParams rp = rope_params(*rope);
+  if (!rope_shape_supported(d, H, rp)) return fail(DSA_ERR_UNSUPPORTED, "unsupported RoPE shape (H_I %d, d_I %d)", H, d);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  Ctx* c = nullptr;
+  dsa_status_t st = get_ctx(stream, &c);
+  if (st != DSA_OK) return st;
+  DSA_CUDA_TRY(launch_rope_queries(q_src, src_dtype == DSA_F32, T, H, d, positions, rp, dst_dtype == DSA_FP8_E4M3,
+                                   q_dst, q_scale, stream),
+               "RoPE query kernel launch");
+  ++g_launches;
   return DSA_OK;
 }
 

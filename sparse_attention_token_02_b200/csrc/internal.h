@@ -114,6 +114,22 @@ cudaError_t launch_topk_stream(const TopkArgs& a, cudaStream_t stream);
 // Rows with at most top_k candidates: every causal position, then padding.
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream);
 
+// Rotary embedding fused into the key append and the query quantisation.
+constexpr int kRopeMaxPairs = 64;      // rope_dim <= 128
+struct RopeParams {
+  int32_t rope_dim;      // leading values of each vector that rotate (even)
+  int32_t interleaved;   // 1: pairs (2i, 2i+1); 0: pairs (i, i + rope_dim / 2)
+  double base;           // theta_i = position * base^(-2 i / rope_dim)
+  double inv_freq[kRopeMaxPairs];   // base^(-2 i / rope_dim), filled by the host
+};
+bool rope_shape_supported(int32_t d, int32_t H, const RopeParams& r);
+cudaError_t launch_rope_append(const void* src, int src_is_f32, int64_t rows, int32_t d, const int64_t* dst_rows,
+                               const int32_t* positions, int64_t capacity, const RopeParams& r, int fp8, void* cache,
+                               float* scale, int* err, cudaStream_t stream);
+cudaError_t launch_rope_queries(const void* src, int src_is_f32, int64_t T, int32_t H, int32_t d,
+                                const int32_t* positions, const RopeParams& r, int fp8, void* dst, float* scale,
+                                cudaStream_t stream);
+
 // After the selection: latent-row gather, int64 cache rows, sorted order.
 bool gather_row_bytes_supported(int32_t row_bytes);
 int sort_selection_max();

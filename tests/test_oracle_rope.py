@@ -44,10 +44,10 @@ def test_relative_position_and_norms(interleaved):
     for p, s in [(10, 3), (107, 100), (7, 0)]:
         a = R.rope_rows(q, np.array([p]), 16, interleaved=interleaved)
         b = R.rope_rows(k, np.array([s]), 16, interleaved=interleaved)
-        dots.append(float(a @ b.T))
+        dots.append((a @ b.T).item())
         np.testing.assert_allclose(np.linalg.norm(a), np.linalg.norm(q), rtol=1e-14)
     np.testing.assert_allclose(dots, dots[0], rtol=1e-12)
-    assert not math.isclose(dots[0], float(q @ k.T), rel_tol=1e-6)
+    assert not math.isclose(dots[0], (q @ k.T).item(), rel_tol=1e-6)
 
 
 def test_heads_share_the_token_angle():
