@@ -11,7 +11,11 @@ Modules
 fp8_e4m3   OCP FP8 E4M3 codec (decode table, RNE + satfinite encode) and the
            per-row absmax quantiser.
 indexer    scores I[t,s], causal mask, top-k with a fixed tie-break, and the
-           prefill / decode drivers over ragged sequences.
+           prefill / decode drivers over ragged sequences (also over an
+           m-compressed key cache).
+rope       the rotary embedding applied to indexer keys and queries.
+after_select  what consumers do with a selection: latent-row gather, int64
+           cache rows, sorted order.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against closed forms,
 hand-summed literals, invariants, brute force on tiny rows, and (for the codec)

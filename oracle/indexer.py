@@ -126,3 +126,40 @@ def decode_oracle(q, k_seqs, w, seq_lens, q_len: int, top_k: int, rows=None,
     """
     q_lens = [int(q_len)] * len(seq_lens)
     return prefill_oracle(q, k_seqs, w, seq_lens, q_lens, top_k, rows=rows, keep_scores=keep_scores)
+
+
+def compressed_visible(position: int, m: int) -> int:
+    """Complete blocks of m tokens a query at token position p sees: floor((p + 1) / m).
+
+    Page "DeepSeek ... Lightning Indexer ... Lookahead Sparse Attention" (the agidaily
+    survey), §三 CSA: every m consecutive tokens' cache entries are merged into one entry and
+    the indexer scores those block entries instead of the raw tokens; the most recent tokens
+    are covered by a separate sliding-window branch.  Reading: a block's entry exists once
+    its m tokens are all in the cache, so the still-open block of the query is not scored.
+    """
+    return (int(position) + 1) // int(m)
+
+
+def decode_compressed_oracle(q, kc_seqs, w, seq_lens, q_lens, m: int, top_k: int) -> dict:
+    """Decode over an m-compressed key cache.
+
+    kc_seqs[b]: [floor(seq_lens[b] / m), d] fp64 compressed keys of sequence b (block j covers
+    tokens j*m .. j*m + m - 1); seq_lens / q_lens in tokens, queries at the last q_lens
+    positions.  Query r at position p scores blocks 0 .. floor((p+1)/m) - 1 (same formula as
+    row_scores) and keeps the top_k blocks.  Returns {"pos", "visible", "idx", "score"}.
+    """
+    seq_lens = [int(x) for x in seq_lens]
+    q_lens = [int(x) for x in q_lens]
+    row_seq = np.repeat(np.arange(len(seq_lens)), q_lens)
+    row_pos = np.concatenate([query_positions(L, n) for L, n in zip(seq_lens, q_lens)])
+    T = row_pos.size
+    out_idx = np.empty((T, top_k), dtype=np.int32)
+    out_val = np.empty((T, top_k), dtype=np.float64)
+    vis = np.empty(T, dtype=np.int64)
+    for r in range(T):
+        b, p = int(row_seq[r]), int(row_pos[r])
+        nv = compressed_visible(p, m)
+        vis[r] = nv
+        s_row = row_scores(q[r], kc_seqs[b][:nv], w[r]) if nv > 0 else np.zeros(0)
+        out_idx[r], out_val[r] = topk_row(s_row, top_k)
+    return {"pos": row_pos, "visible": vis, "idx": out_idx, "score": out_val}

@@ -19,6 +19,7 @@ import pytest
 
 import oracle
 from oracle import decode_oracle, prefill_oracle, row_scores, topk_row
+from oracle import indexer as O
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -255,3 +256,41 @@ def test_planted_causal_off_by_one_fails_a_pin():
     # strict s < t would drop the diagonal: row 2 would lose its best key (s=2, score 1.0)
     strict = [row_scores(q[t], k[:t], w[t]) for t in range(3)]
     assert strict[2].tolist() != c["scores"][2]
+
+
+# ----------------------------------------------------------------------------- m-compressed cache
+
+def test_compressed_visible_at_block_boundaries():
+    # m = 4: the block of tokens 0..3 exists from position 3 on
+    assert [O.compressed_visible(p, 4) for p in (0, 2, 3, 6, 7, 8, 11)] == [0, 0, 1, 1, 2, 2, 3]
+    assert [O.compressed_visible(p, 1) for p in (0, 5)] == [1, 6]
+
+
+def test_compressed_decode_with_m_1_is_plain_decode():
+    rng = np.random.default_rng(5)
+    lens, q_lens, H, d, k = (40, 13), (2, 1), 3, 8, 6
+    keys = [rng.standard_normal((L, d)) for L in lens]
+    q = rng.standard_normal((sum(q_lens), H, d))
+    w = rng.random((sum(q_lens), H))
+    a = O.decode_compressed_oracle(q, keys, w, lens, q_lens, 1, k)
+    b = O.prefill_oracle(q, keys, w, lens, q_lens, k)
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["score"], b["score"])
+
+
+def test_compressed_decode_hand_case():
+    # H = 1, d = 1, w = 1: I[s] = ReLU(q k_s) / 1.  m = 2, sequence of 7 tokens -> 3 blocks.
+    kc = [np.array([[1.0], [3.0], [-2.0]])]
+    q = np.array([[[2.0]], [[2.0]]])
+    w = np.ones((2, 1))
+    res = O.decode_compressed_oracle(q, kc, w, (7,), (2,), 2, 2)
+    # position 5 sees blocks 0..2 (floor(6/2) = 3); position 6 also 3 (block 3 not complete)
+    assert res["visible"].tolist() == [3, 3]
+    assert res["idx"][0].tolist() == [1, 0] and res["score"][0].tolist() == [6.0, 2.0]
+    # with q_len 1 at the end of a 6-token sequence, floor(6/2) = 3 blocks as well
+    res = O.decode_compressed_oracle(q[:1], kc, w[:1], (6,), (1,), 2, 4)
+    assert res["idx"][0].tolist() == [1, 0, 2, -1]
+    assert res["score"][0].tolist() == [6.0, 2.0, 0.0, -np.inf]
+    # a 1-token sequence sees no block at m = 2
+    res = O.decode_compressed_oracle(q[:1], [np.zeros((0, 1))], w[:1], (1,), (1,), 2, 2)
+    assert res["visible"].tolist() == [0] and res["idx"][0].tolist() == [-1, -1]
