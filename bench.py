@@ -355,6 +355,46 @@ def rope_timings(api, stream, dev, reps=10):
     return out
 
 
+def compressed_timings(api, hx, stream, dev, m=4, reps=10):
+    """Decode over an m-compressed key cache with the decode batch's shape (block keys
+    synthetic N(0, 1) bf16, one row per m tokens); CUDA events around each call after a
+    256 MB L2-evicting read."""
+    import torch
+    wl = hx.wl
+    blocks = [L // m for L in wl.seq_lens]
+    base = np.concatenate([[0], np.cumsum(blocks)[:-1]]).astype(np.int64)
+    with torch.cuda.stream(stream):
+        cache = api.IndexerKCache.empty(int(sum(blocks)), wl.d, False, device=dev)
+        keys = torch.randn(int(sum(blocks)), wl.d, device=dev).to(torch.bfloat16)
+        api.dsa_indexer_kcache_append(cache, keys, torch.arange(int(sum(blocks)), dtype=torch.int64, device=dev),
+                                      stream=stream)
+        flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        oi = torch.empty(wl.total_q, wl.top_k, dtype=torch.int32, device=dev)
+        os_ = torch.empty(wl.total_q, wl.top_k, dtype=torch.float32, device=dev)
+    call = lambda: api.dsa_indexer_decode_compressed(hx.q, cache, hx.w, hx.seq_lens, hx.q_lens, m, wl.top_k,
+                                                     k_base=base, out_idx=oi, out_score=os_, stream=stream)
+    call()
+    total = 0.0
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            flush.max()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        stream.synchronize()
+        total += e0.elapsed_time(e1)
+    api.dsa_check_device_errors(stream)
+    ms = total / reps
+    pairs = sum((L - n + j + 1) // m for L, n in zip(wl.seq_lens, wl.q_lens) for j in range(n))
+    kbytes = int(sum(blocks)) * wl.d * 2
+    hbm = peaks()["hbm"]
+    del cache, keys, flush
+    return {"m": m, "ms": ms, "pairs": pairs, "pairs_per_s": pairs / (ms * 1e-3),
+            "key_bytes": kbytes, "frac_of_hbm": kbytes / (ms * 1e-3) / 1e9 / hbm,
+            "note": "eager call (logits + top-k), one single-query decode row per query"}
+
+
 class Harness:
     """Device state and one step of the hot path for a workload.
 
@@ -579,6 +619,7 @@ def run_ours(args):
     # attention makes and the sorted order, each launch timed alone after an L2 flush
     after = after_select_timings(api, hx, stream, dev) if hx.decode else None
     rope = rope_timings(api, stream, dev) if hx.decode else None
+    comp = compressed_timings(api, hx, stream, dev) if hx.decode and not hx.fp8 else None
 
     # roofline of the dominant kernel (the logits kernel)
     pk = peaks()
@@ -627,6 +668,8 @@ def run_ours(args):
             line["after_select"] = after
         if rope is not None:
             line["rope_fused"] = rope
+        if comp is not None:
+            line["compressed_decode"] = comp
         print(json.dumps(line), flush=True)
     del graph
     if world > 1:

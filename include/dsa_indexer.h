@@ -216,6 +216,25 @@ DSA_API dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const dsa_
                                                 float* out_score, int32_t* fault, void* stream);
 
 /*
+ * Decode over an m-compressed indexer key cache (the agidaily survey of DSA and its
+ * successors, §三 CSA: every m consecutive tokens' entries are merged into one, and the
+ * indexer scores those block entries; the merge itself is learned and is the caller's).
+ *   kc      cache of compressed keys: row k_base[b] + j holds block j of sequence b,
+ *           i.e. tokens j*m .. j*m + m - 1 (bf16 or FP8 + scale, as for dsa_indexer_decode)
+ *   batch   seq_lens / q_lens in TOKENS; the queries sit at the last q_lens positions;
+ *           k_base = first compressed row of each sequence (NULL: sequences' blocks packed
+ *           back to back from row 0, floor(seq_len / m) rows each)
+ *   m       tokens per block (>= 1; m = 1 is dsa_indexer_decode)
+ * A query at token position p sees the complete blocks j < floor((p + 1) / m): its own
+ * still-open block is not scored (the sliding-window branch covers it).  out_idx holds
+ * block indices j, out_score their scores; a query that sees no block gets only -1 / -inf.
+ * Every q_lens[b] is at most 4 and every query is scored as its own single-query decode row.
+ */
+DSA_API dsa_status_t dsa_indexer_decode_compressed(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                                   const dsa_batch_t* batch, int32_t m, int32_t top_k,
+                                                   int32_t* out_idx, float* out_score, void* stream);
+
+/*
  * Rotary position embedding of indexer keys and queries, fused into the cache append and
  * the query quantisation (page "Study MLA Indexer", section 数学流: the key is RoPE'd, then
  * quantised and written to the indexer K cache; the query is RoPE'd).  The pages give no

@@ -197,6 +197,24 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
                                               _ptr(out_score_host), _stream(stream)))
 
 
+def dsa_indexer_decode_compressed(q, cache: IndexerKCache, w, seq_lens, q_lens, m, top_k, q_scale=None,
+                                  k_base=None, out_idx=None, out_score=None, stream=None):
+    """Decode over an m-compressed key cache (block j of sequence b at cache row k_base[b] + j);
+    seq_lens / q_lens in tokens.  Returns (block indices int32 [T, k], scores fp32 [T, k])."""
+    b = _HostBatch(seq_lens, q_lens, k_base)
+    T = b.total_q
+    _require_cuda(w)
+    if out_idx is None:
+        out_idx = torch.empty(T, top_k, dtype=torch.int32, device=q.device)
+    if out_score is None:
+        out_score = torch.empty(T, top_k, dtype=torch.float32, device=q.device)
+    _require_cuda(out_idx, out_score)
+    qq, kc = _query(q, q_scale), cache.c()
+    check(_lib.load().dsa_indexer_decode_compressed(ctypes.byref(qq), ctypes.byref(kc), _ptr(w), ctypes.byref(b.c),
+                                                    int(m), top_k, _ptr(out_idx), _ptr(out_score), _stream(stream)))
+    return out_idx, out_score
+
+
 def _rope(d, rope_dim, base, interleaved):
     from ._lib import Rope
     return Rope(d if rope_dim is None else int(rope_dim), 1 if interleaved else 0, float(base))

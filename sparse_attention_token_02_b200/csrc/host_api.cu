@@ -899,6 +899,58 @@ dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* k
   return DSA_OK;
 }
 
+dsa_status_t dsa_indexer_decode_compressed(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                           const dsa_batch_t* batch, int32_t m, int32_t top_k, int32_t* out_idx,
+                                           float* out_score, void* stream_v) {
+  g_last_error.clear();
+  if (!q || !kc || !w || !batch || !out_idx || !out_score) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (m < 1 || top_k < 1) return fail(DSA_ERR_INVALID_ARG, "m and top_k must be >= 1");
+  if (batch->num_seqs < 0 || (batch->num_seqs > 0 && (!batch->seq_lens || !batch->q_lens)))
+    return fail(DSA_ERR_INVALID_ARG, "decode needs batch.seq_lens and batch.q_lens");
+  if (q->dtype != DSA_BF16 && q->dtype != DSA_FP8_E4M3) return fail(DSA_ERR_INVALID_ARG, "q->dtype must be DSA_BF16 or DSA_FP8_E4M3");
+  // every query becomes a single-query decode row over its visible blocks
+  std::vector<int32_t> vis;
+  std::vector<int64_t> base;
+  int64_t packed = 0;
+  for (int b = 0; b < batch->num_seqs; ++b) {
+    const int32_t L = batch->seq_lens[b], n = batch->q_lens[b];
+    if (L < 0 || n < 0 || n > L || n > 4) return fail(DSA_ERR_INVALID_ARG, "sequence %d: need 0 <= q_len <= min(4, seq_len)", b);
+    const int64_t kb = batch->k_base ? batch->k_base[b] : packed;
+    packed += L / m;
+    for (int32_t j = 0; j < n; ++j) {
+      vis.push_back((L - n + j + 1) / m);
+      base.push_back(kb);
+    }
+  }
+  const int64_t T = static_cast<int64_t>(vis.size());
+  const size_t q_row = size_t(q->H_I) * q->d_I * (q->dtype == DSA_FP8_E4M3 ? 1 : 2);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  dsa_status_t st;
+  // runs of rows that see at least one block go through the decode path; the rest are padding
+  for (int64_t r0 = 0; r0 < T;) {
+    int64_t r1 = r0;
+    const bool any = vis[r0] > 0;
+    while (r1 < T && (vis[r1] > 0) == any) ++r1;
+    if (any) {
+      const std::vector<int32_t> ones(size_t(r1 - r0), 1);
+      dsa_batch_t pb{static_cast<int32_t>(r1 - r0), vis.data() + r0, ones.data(), base.data() + r0};
+      dsa_query_t qr = *q;
+      qr.data = static_cast<const char*>(q->data) + r0 * q_row;
+      qr.scale = q->scale ? q->scale + r0 : nullptr;
+      if ((st = dsa_indexer_decode(&qr, kc, w + r0 * q->H_I, &pb, top_k, out_idx + r0 * top_k,
+                                   out_score + r0 * top_k, stream_v)) != DSA_OK)
+        return st;
+    } else {
+      const int64_t cnt = (r1 - r0) * top_k;
+      DSA_CUDA_TRY(cudaMemsetAsync(out_idx + r0 * top_k, 0xFF, size_t(cnt) * sizeof(int32_t), stream), "cudaMemsetAsync");
+      DSA_CUDA_TRY(launch_fill_f32(out_score + r0 * top_k, cnt, -INFINITY, stream), "fill kernel launch");
+      ++g_launches;
+    }
+    r0 = r1;
+  }
+  return DSA_OK;
+}
+
 dsa_status_t dsa_indexer_kcache_append_rope(const dsa_kcache_t* kc, const void* k_new, dsa_dtype_t src_dtype,
                                             const int64_t* dst_rows, const int32_t* positions, int32_t n,
                                             const dsa_rope_t* rope, void* stream_v) {

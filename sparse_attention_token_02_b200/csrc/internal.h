@@ -130,6 +130,8 @@ cudaError_t launch_rope_queries(const void* src, int src_is_f32, int64_t T, int3
                                 const int32_t* positions, const RopeParams& r, int fp8, void* dst, float* scale,
                                 cudaStream_t stream);
 
+cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
+
 // After the selection: latent-row gather, int64 cache rows, sorted order.
 bool gather_row_bytes_supported(int32_t row_bytes);
 int sort_selection_max();

@@ -144,6 +144,12 @@ __global__ void __launch_bounds__(kSortThreads) sort_selection_kernel(int32_t* _
   }
 }
 
+__global__ void __launch_bounds__(256) fill_f32_kernel(float* __restrict__ p, int64_t n, float v) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = v;
+}
+
 cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -157,6 +163,13 @@ cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t stream, cudaLa
 }
 
 }  // namespace
+
+cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256;
+  fill_f32_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, stream>>>(p, n, v);
+  return cudaGetLastError();
+}
 
 bool gather_row_bytes_supported(int32_t row_bytes) {
   return row_bytes > 0 && row_bytes % 16 == 0 && row_bytes / 16 <= kMaxRowVecs;
