@@ -721,6 +721,11 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     s.row_ctr = reinterpret_cast<uint32_t*>(wsb + wl.ctr);
     s.cand_key = reinterpret_cast<uint32_t*>(wsb + wl.cand_key);
     s.cand_idx = reinterpret_cast<int32_t*>(wsb + wl.cand_idx);
+    if (fp8) {
+      // the FP8 logits epilogue leaves the coarse histograms to a pass over the score rows
+      DSA_CUDA_TRY(launch_row_hist(s, stream), "row histogram launch");
+      ++g_launches;
+    }
     DSA_CUDA_TRY(launch_topk_stream(s, stream), "top-k (streaming) launch");
     ++g_launches;
   }

@@ -111,6 +111,9 @@ cudaError_t launch_topk_rows(const TopkArgs& a, cudaStream_t stream);
 // Rows whose coarse histogram the logits epilogue built: one CTA per chunk of kStreamChunk
 // keys, the last CTA of a row finishing the selection inside the threshold bin.
 cudaError_t launch_topk_stream(const TopkArgs& a, cudaStream_t stream);
+// Coarse row histograms from the score rows (decode configurations whose logits epilogue
+// does not count them), one CTA per streaming chunk; row_hist must start zeroed.
+cudaError_t launch_row_hist(const TopkArgs& a, cudaStream_t stream);
 // Rows with at most top_k candidates: every causal position, then padding.
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream);
 

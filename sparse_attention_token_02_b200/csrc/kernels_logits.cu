@@ -84,7 +84,10 @@ struct Cfg {
   // latency, sets the pace (prefill): then they leave the issue slots to the epilogue
   static constexpr bool PIPE_SLEEP = NG > 1;
   // decode configurations can bin every row for the top-k (prefill ones compile no such code)
-  static constexpr bool HIST = NG == 1;
+  // bf16 decode configurations bin every row for the top-k in the epilogue, where the HBM-bound
+  // loop leaves the epilogue slack; FP8 decode (twice the keys per byte) leaves it none, so its
+  // rows are binned by a separate pass over the score rows, and prefill configurations not at all
+  static constexpr bool HIST = NG == 1 && !FP8;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + STAGES * K_TILE_BYTES;
@@ -93,16 +96,8 @@ struct Cfg {
   static constexpr int OFF_W = OFF_Q + Q_BYTES;
   static constexpr int W_WARP_FLOATS = NT * H;
   static constexpr int OFF_ROW = OFF_W + NE * W_WARP_FLOATS * 4;
-  // FP8 decode, where it fits: the coarse histogram of the item's query rows is counted in
-  // shared memory (plain shared atomics in the per-tile chain) and flushed to the global rows
-  // at the end of each item; elsewhere lanes are merged and counted straight into HBM.
-  static constexpr int OFF_HIST = (OFF_ROW + NE * NT * 8 + 15) / 16 * 16;
-  static constexpr int HIST_SMEM_BYTES = NT * kHistBins * 4;
-  static constexpr int BASE_BARS = 2 * STAGES + 2 + 2 * NBUF + 1;
-  static constexpr bool HIST_SMEM =
-      HIST && FP8 && OFF_HIST + HIST_SMEM_BYTES + (BASE_BARS + 2) * 8 + 16 + 1024 <= 227 * 1024;
-  static constexpr int OFF_BAR = ((HIST_SMEM ? OFF_HIST + HIST_SMEM_BYTES : OFF_ROW + NE * NT * 8) + 7) / 8 * 8;
-  static constexpr int NUM_BARS = BASE_BARS + (HIST_SMEM ? 2 : 0);
+  static constexpr int OFF_BAR = (OFF_ROW + NE * NT * 8 + 7) / 8 * 8;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 * NBUF + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // + alignment slack; at least 120 KB so that one CTA holds an SM (and all its TMEM)
   static constexpr int SMEM_RAW = OFF_MISC + 16 + 1024;
@@ -223,9 +218,6 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
   uint64_t* acc_full = q_full + 2;
   uint64_t* acc_empty = acc_full + C::NBUF;
   uint64_t* drain = acc_empty + C::NBUF;
-  uint64_t* hist_done = drain + 1;            // HIST_SMEM: every epilogue warp finished the item
-  uint64_t* flush_done = drain + 2;           // HIST_SMEM: the item's counts are in HBM, bins zero
-  uint32_t* shist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -248,10 +240,6 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
       mbar_init(&acc_empty[b], C::NEG);
     }
     mbar_init(drain, 1);
-    if constexpr (C::HIST_SMEM) {
-      mbar_init(hist_done, C::NE);
-      mbar_init(flush_done, C::NE);
-    }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_k);
@@ -261,8 +249,6 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if constexpr (C::HIST_SMEM)
-    for (int i = threadIdx.x; i < C::HIST_SMEM_BYTES / 4; i += C::THREADS) shist[i] = 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -407,17 +393,12 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
     float* wq = reinterpret_cast<float*>(smem + C::OFF_W) + ew * C::W_WARP_FLOATS;
     int64_t* rowoff = reinterpret_cast<int64_t*>(smem + C::OFF_ROW) + ew * C::NT;
     uint32_t acc_iter = 0;
-    uint32_t hist_phase = 0;
     bool ok = true;
     for (int it = item_begin; it < item_end && ok; ++it) {
       const LogitsItem wi = args.items[it];
       // counts score v of the item's query j in its row's coarse histogram; all lanes together
       auto hist_count = [&](int j, float v, bool valid) {
-        if constexpr (C::HIST_SMEM) {
-          if (valid) atomicAdd(shist + j * kHistBins + (order_key(__float_as_uint(v)) >> kHistShift), 1u);
-        } else {
-          coarse_hist_add(args.row_hist + static_cast<int64_t>(wi.q_row0 + j) * kHistBins, v, valid);
-        }
+        coarse_hist_add(args.row_hist + static_cast<int64_t>(wi.q_row0 + j) * kHistBins, v, valid);
       };
       __syncwarp();                           // this warp is done with the previous item's copies
       for (int i = lane; i < wi.n_tok * C::H; i += 32) {
@@ -575,27 +556,6 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
           st_[4] += clock64() - tc0_;
 #endif
           if (lane == 0) mbar_arrive(&acc_empty[b]);
-        }
-      }
-      if constexpr (C::HIST_SMEM) {
-        if (ok && args.row_hist) {
-          // every epilogue warp has counted the item; flush its rows' bins, then zero them
-          // for the next item (both waits bounded, like every other wait of the kernel)
-          __syncwarp();
-          if (lane == 0) mbar_arrive(hist_done);
-          if (!mbar_wait(hist_done, hist_phase & 1, abort_flag)) { ok = false; break; }
-          for (int i = ew * 32 + lane; i < wi.n_tok * kHistBins; i += C::NE * 32) {
-            const uint32_t c = shist[i];
-            if (c) {
-              const int j = i / kHistBins;
-              atomicAdd(args.row_hist + static_cast<int64_t>(wi.q_row0 + j) * kHistBins + (i - j * kHistBins), c);
-              shist[i] = 0u;
-            }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(flush_done);
-          if (!mbar_wait(flush_done, hist_phase & 1, abort_flag)) { ok = false; break; }
-          ++hist_phase;
         }
       }
     }

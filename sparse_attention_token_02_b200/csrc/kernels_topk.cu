@@ -1036,6 +1036,41 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
   }
 }
 
+// Coarse row histograms for decode configurations whose logits epilogue does not count
+// them (FP8): one CTA per streaming chunk of kStreamChunk scores counts its keys' top bits in
+// a shared histogram and adds the non-zero bins to the row's global histogram.
+constexpr int kRowHistThreads = 256;
+static_assert(kStreamChunk % (4 * kRowHistThreads) == 0, "whole float4 per thread and pass");
+
+__global__ void __launch_bounds__(kRowHistThreads) row_hist_kernel(const TopkArgs a) {
+  __shared__ uint32_t h[kHistBins];
+  const int tid = threadIdx.x;
+  for (int b = tid; b < kHistBins; b += kRowHistThreads) h[b] = 0u;
+  const TopkChunk ch = a.chunks[blockIdx.x];
+  const float* src = a.scores + a.row_off[ch.row];
+  __syncthreads();
+  grid_dependency_wait();                     // the scores come from the previous kernel
+  constexpr int kPer = kStreamChunk / (4 * kRowHistThreads);
+  float4 f[kPer];
+#pragma unroll
+  for (int v = 0; v < kPer; ++v) {            // every load in flight before any is counted
+    const int i = ch.begin + (v * kRowHistThreads + tid) * 4;
+    f[v] = i < ch.end ? __ldcg(reinterpret_cast<const float4*>(src + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int v = 0; v < kPer; ++v) {
+    const int i = ch.begin + (v * kRowHistThreads + tid) * 4;
+    const float fv[4] = {f[v].x, f[v].y, f[v].z, f[v].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (i + e < ch.end) atomicAdd(&h[float_to_key(fv[e]) >> kHistShift], 1u);
+  }
+  __syncthreads();
+  uint32_t* row_hist = const_cast<uint32_t*>(a.row_hist) + static_cast<int64_t>(ch.row) * kHistBins;
+  for (int b = tid; b < kHistBins; b += kRowHistThreads)
+    if (h[b]) atomicAdd(row_hist + b, h[b]);
+}
+
 // Rows whose whole causal history fits in top_k: every position, then -1 / -inf.
 __global__ void __launch_bounds__(256) topk_short_kernel(const TopkArgs a) {
   grid_dependency_wait();                     // the scores come from the previous kernel
@@ -1134,6 +1169,20 @@ cudaError_t launch_topk_rows(const TopkArgs& a, cudaStream_t stream) {
     if (dev < 64) configured |= 1ull << dev;
   }
   return cudaLaunchKernelEx(&cfg, topk_row_kernel, a);
+}
+
+cudaError_t launch_row_hist(const TopkArgs& a, cudaStream_t stream) {
+  if (a.n_chunks <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.n_chunks), 1, 1);
+  cfg.blockDim = dim3(kRowHistThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, row_hist_kernel, a);
 }
 
 cudaError_t launch_topk_short(const TopkArgs& a, cudaStream_t stream) {
