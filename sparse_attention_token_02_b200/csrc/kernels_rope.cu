@@ -34,34 +34,41 @@ __device__ __forceinline__ float2 pair_cos_sin(int i, int32_t p, const RopeParam
   return make_float2(c, s);
 }
 
-// Rotates the EPL values v[] a lane holds (values lane*EPL .. lane*EPL+EPL-1 of a d-vector)
-// with the pairs' (cos, sin) in cs[].
+// The (cos, sin) each of a lane's EPL values rotates with (values lane*EPL .. lane*EPL+EPL-1
+// of a d-vector), read once from cs[] into registers; (1, 0) past rope_dim.
 template <int EPL>
-__device__ __forceinline__ void rope_lane(float (&v)[EPL], int lane, const float2* cs, const RopeParams& r) {
+__device__ __forceinline__ void lane_cos_sin(int lane, const float2* cs, const RopeParams& r, float2 (&t)[EPL]) {
   const int half = r.rope_dim / 2;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int idx = lane * EPL + e;
+    const int pair = r.interleaved ? idx / 2 : (idx < half ? idx : idx - half);
+    t[e] = idx < r.rope_dim ? cs[pair] : make_float2(1.f, 0.f);
+  }
+}
+
+// Rotates the EPL values v[] a lane holds with the lane's (cos, sin) t[].
+template <int EPL>
+__device__ __forceinline__ void rope_lane(float (&v)[EPL], int lane, const float2 (&t)[EPL], const RopeParams& r) {
+  const bool rotates = lane * EPL < r.rope_dim;           // values past rope_dim pass through untouched
   if (r.interleaved) {
 #pragma unroll
-    for (int e = 0; e < EPL; e += 2) {
-      const int i = (lane * EPL + e) / 2;                 // pair index
-      if (2 * i < r.rope_dim) {
-        const float2 t = cs[i];
-        const float a = v[e], b = v[e + 1];
-        v[e] = a * t.x - b * t.y;
-        v[e + 1] = a * t.y + b * t.x;
+    for (int e = 0; e < EPL; e += 2) {                    // pairs (2i, 2i+1) lie inside the lane
+      const float a = v[e], b = v[e + 1];
+      if (rotates) {
+        v[e] = a * t[e].x - b * t[e].y;
+        v[e + 1] = a * t[e].y + b * t[e].x;
       }
     }
   } else {
     // pair (i, i + half): the partner value sits half / EPL lanes away (half % EPL == 0)
+    const int half = r.rope_dim / 2;
     const int lane_off = half / EPL;
+    const bool first = lane * EPL < half;                 // a lane's values all sit on one side
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
-      const int idx = lane * EPL + e;
       const float other = __shfl_xor_sync(0xffffffffu, v[e], lane_off);   // lane_off is a power of two
-      if (idx < r.rope_dim) {
-        const bool first = idx < half;
-        const float2 t = cs[first ? idx : idx - half];
-        v[e] = first ? v[e] * t.x - other * t.y : other * t.y + v[e] * t.x;
-      }
+      if (rotates) v[e] = first ? v[e] * t[e].x - other * t[e].y : other * t[e].y + v[e] * t[e].x;
     }
   }
 }
@@ -148,7 +155,9 @@ rope_append_kernel(const void* __restrict__ src, int src_is_f32, int64_t rows, c
   const int32_t p = positions[row];
   for (int i = lane; i < rp.rope_dim / 2; i += 32) cs[i] = pair_cos_sin(i, p, rp);
   __syncwarp();
-  rope_lane<EPL>(v, lane, cs, rp);
+  float2 t[EPL];
+  lane_cos_sin<EPL>(lane, cs, rp, t);
+  rope_lane<EPL>(v, lane, t, rp);
   if (fp8) {
     float amax = 0.f;
 #pragma unroll
@@ -166,7 +175,7 @@ rope_append_kernel(const void* __restrict__ src, int src_is_f32, int64_t rows, c
 // One CTA per query token: warp w rotates heads w, w + kRopeWarps, ... (at most HPW each);
 // FP8 output shares one scale over all H * d values of the token.
 template <int EPL, int HPW>
-__global__ void __launch_bounds__(kRopeWarps * 32)
+__global__ void __launch_bounds__(kRopeWarps * 32, 4)
 rope_queries_kernel(const void* __restrict__ src, int src_is_f32, int32_t H, const int32_t* __restrict__ positions,
                     RopeParams rp, int fp8, void* __restrict__ dst, float* __restrict__ scale) {
   launch_dependents();
@@ -185,12 +194,14 @@ rope_queries_kernel(const void* __restrict__ src, int src_is_f32, int32_t H, con
   const int32_t p = positions[t];
   for (int i = threadIdx.x; i < rp.rope_dim / 2; i += kRopeWarps * 32) cs[i] = pair_cos_sin(i, p, rp);
   __syncthreads();
+  float2 tcs[EPL];                                      // the same for every head of the token
+  lane_cos_sin<EPL>(lane, cs, rp, tcs);
   float amax = 0.f;
 #pragma unroll
   for (int u = 0; u < kMaxHeadsPerWarp; ++u) {
     const int h = warp + u * kRopeWarps;
     if (h < H) {
-      rope_lane<EPL>(v[u], lane, cs, rp);
+      rope_lane<EPL>(v[u], lane, tcs, rp);
 #pragma unroll
       for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
     }
