@@ -318,6 +318,15 @@ DSA_API dsa_status_t dsa_set_workspace(void* ptr, size_t bytes, void* stream);
 DSA_API dsa_status_t dsa_check_device_errors(void* stream);
 
 /*
+ * Self-test of failure detection: one kernel waits, with the same bounded wait every kernel
+ * of this library uses, on a barrier that nothing completes, giving up after limit_cycles SM
+ * clock cycles (1 .. 2e9).  The expiry is recorded like any device fault: the next
+ * dsa_check_device_errors(stream) returns DSA_ERR_DEVICE_CHECK ("a bounded wait expired")
+ * and clears it; the stream stays usable.
+ */
+DSA_API dsa_status_t dsa_selftest_wait_expiry(int64_t limit_cycles, void* stream);
+
+/*
  * Profiling hook.  Registers three cudaEvent_t for the calling thread (NULL
  * clears them): every later prefill / decode / scores call on this thread
  * records ev_begin right before its logits kernel, ev_mid right after it and

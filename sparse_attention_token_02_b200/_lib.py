@@ -35,6 +35,7 @@ EXPORTED = (
     "dsa_indexer_workspace_bytes",
     "dsa_set_workspace",
     "dsa_check_device_errors",
+    "dsa_selftest_wait_expiry",
     "dsa_set_profile_events",
     "dsa_kernel_launch_count",
     "dsa_get_last_error",
@@ -113,6 +114,8 @@ def load() -> ctypes.CDLL:
     lib.dsa_set_workspace.restype = st
     lib.dsa_check_device_errors.argtypes = [V]
     lib.dsa_check_device_errors.restype = st
+    lib.dsa_selftest_wait_expiry.argtypes = [I64, V]
+    lib.dsa_selftest_wait_expiry.restype = st
     lib.dsa_set_profile_events.argtypes = [V, V, V]
     lib.dsa_set_profile_events.restype = st
     lib.dsa_kernel_launch_count.argtypes = []

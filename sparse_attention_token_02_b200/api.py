@@ -197,6 +197,12 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
                                               _ptr(out_score_host), _stream(stream)))
 
 
+def dsa_selftest_wait_expiry(limit_cycles=100000, stream=None):
+    """Run the bounded-wait self-test (a wait on a barrier nothing completes, given up after
+    limit_cycles); the expiry then shows in dsa_check_device_errors."""
+    check(_lib.load().dsa_selftest_wait_expiry(int(limit_cycles), _stream(stream)))
+
+
 def dsa_indexer_decode_compressed(q, cache: IndexerKCache, w, seq_lens, q_lens, m, top_k, q_scale=None,
                                   k_base=None, out_idx=None, out_score=None, stream=None):
     """Decode over an m-compressed key cache (block j of sequence b at cache row k_base[b] + j);

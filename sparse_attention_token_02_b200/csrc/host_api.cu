@@ -956,6 +956,18 @@ dsa_status_t dsa_indexer_decode_compressed(const dsa_query_t* q, const dsa_kcach
   return DSA_OK;
 }
 
+dsa_status_t dsa_selftest_wait_expiry(int64_t limit_cycles, void* stream_v) {
+  g_last_error.clear();
+  if (limit_cycles < 1 || limit_cycles > 2000000000LL) return fail(DSA_ERR_INVALID_ARG, "limit_cycles must be in 1 .. 2e9");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  Ctx* c = nullptr;
+  dsa_status_t st = get_ctx(stream, &c);
+  if (st != DSA_OK) return st;
+  DSA_CUDA_TRY(launch_wait_expiry(limit_cycles, c->d_err, stream), "self-test kernel launch");
+  ++g_launches;
+  return DSA_OK;
+}
+
 dsa_status_t dsa_indexer_kcache_append_rope(const dsa_kcache_t* kc, const void* k_new, dsa_dtype_t src_dtype,
                                             const int64_t* dst_rows, const int32_t* positions, int32_t n,
                                             const dsa_rope_t* rope, void* stream_v) {

@@ -134,6 +134,7 @@ cudaError_t launch_rope_queries(const void* src, int src_is_f32, int64_t T, int3
                                 cudaStream_t stream);
 
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
+cudaError_t launch_wait_expiry(long long limit_cycles, int* err, cudaStream_t stream);
 
 // After the selection: latent-row gather, int64 cache rows, sorted order.
 bool gather_row_bytes_supported(int32_t row_bytes);

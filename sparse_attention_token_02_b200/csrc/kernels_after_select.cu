@@ -150,6 +150,23 @@ __global__ void __launch_bounds__(256) fill_f32_kernel(float* __restrict__ p, in
     p[i] = v;
 }
 
+// Self-test of the bounded wait every kernel of the library uses: one CTA waits on an
+// mbarrier that nothing arrives at, with a short limit; the wait must expire, raise the CTA's
+// abort flag and let the kernel record DSA_DEVERR_TIMEOUT and return.
+__global__ void wait_expiry_kernel(long long limit_cycles, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool done = mbar_wait(&bar, 0, &abort_flag, limit_cycles);   // no arrival ever comes
+  __syncthreads();
+  if (threadIdx.x == 0 && !done && abort_flag) record_error(err, DSA_DEVERR_TIMEOUT, static_cast<int>(blockIdx.x));
+}
+
 cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -176,6 +193,11 @@ bool gather_row_bytes_supported(int32_t row_bytes) {
 }
 
 int sort_selection_max() { return kSortMax; }
+
+cudaError_t launch_wait_expiry(long long limit_cycles, int* err, cudaStream_t stream) {
+  wait_expiry_kernel<<<1, 64, 0, stream>>>(limit_cycles, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gather_rows(const void* src, int64_t src_rows, int32_t row_bytes, const int32_t* idx,
                                const int64_t* row_base, int64_t rows, int32_t top_k, void* dst, int* err, int sms,

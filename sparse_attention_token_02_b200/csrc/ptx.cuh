@@ -80,19 +80,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false if the
-// wait ran past kWaitLimitCycles or another role raised *abort (volatile smem).
+// wait ran past limit_cycles (default kWaitLimitCycles, about a second) or another role
+// raised *abort (volatile smem); on its own expiry it raises *abort itself.
 #ifndef DSA_SPIN_BACKOFF_NS
 #define DSA_SPIN_BACKOFF_NS 0
 #endif
 template <bool kSleep = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long limit_cycles = kWaitLimitCycles) {
   if (mbar_try_wait<kSleep>(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (!kSleep && DSA_SPIN_BACKOFF_NS > 0) __nanosleep(DSA_SPIN_BACKOFF_NS);   // fewer issue slots spent spinning
     if (mbar_try_wait<kSleep>(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit_cycles) {
       *abort = 1;
       return false;
     }

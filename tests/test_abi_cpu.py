@@ -120,3 +120,9 @@ def test_workspace_bytes_grows_with_the_triangle(lib):
     a = lib.dsa_indexer_workspace_bytes(ctypes.byref(q), ctypes.byref(small), 2048)
     c = lib.dsa_indexer_workspace_bytes(ctypes.byref(q), ctypes.byref(big), 2048)
     assert a > 1000 * 1001 // 2 * 4 and c > 4000 * 4001 // 2 * 4 and c > a
+
+
+def test_wait_expiry_self_test_checks_its_limit(lib):
+    for bad in (0, -5, 3_000_000_000):
+        st = lib.dsa_selftest_wait_expiry(bad, None)
+        assert _lib.STATUS_NAMES[st] == "DSA_ERR_INVALID_ARG", lib.dsa_get_last_error()

@@ -125,6 +125,16 @@ def test_append_out_of_range_row_is_reported_and_skipped():
     api.dsa_check_device_errors()           # the flag was cleared
 
 
+def test_bounded_wait_expiry_is_reported_and_the_stream_stays_usable():
+    # the library's bounded wait, on a barrier that nothing completes, with a ~1 ms limit
+    api.dsa_selftest_wait_expiry(2_000_000)
+    with pytest.raises(RuntimeError, match="DEVICE_CHECK.*bounded wait expired"):
+        api.dsa_check_device_errors()
+    api.dsa_check_device_errors()           # the flag was cleared
+    x = torch.arange(1024, dtype=torch.float32, device="cuda")
+    assert float(x.sum()) == 1023 * 1024 / 2
+
+
 # ----------------------------------------------------------------------------- prefill
 
 def test_tiny_workload_all_rows_and_dense_scores():
