@@ -61,6 +61,10 @@ def parse():
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="profiling only: run this many untimed steps of the workload and exit (no JSON line); "
                          "the command ncu wraps to capture single kernels")
+    ap.add_argument("--only", choices=["rope"], default=None,
+                    help="profiling only: time one side section alone (rope: the fused RoPE kernels at prefill "
+                         "size) and print its figures as JSON, without the decode workload")
+    ap.add_argument("--reps", type=int, default=10, help="launches per kernel in --only")
     return ap.parse_args()
 
 
@@ -267,6 +271,12 @@ def profiled_traffic():
         return None
 
 
+# Before a launch timed alone, the GPU spins this many cycles (about 150 us) after the L2
+# flush, so the host has enqueued the start event, the launch and the end event before the
+# device reaches them: the events then bracket device time only, not the host's call overhead.
+_HOST_LEAD_CYCLES = 300_000
+
+
 def after_select_timings(api, hx, stream, dev, reps=10):
     """Latent-row gather (bf16 c^KV, d_c = 512 per cached token, synthetic) at the step's
     selection, and the in-place sort of the selection; CUDA events around each launch.  Before
@@ -284,10 +294,11 @@ def after_select_timings(api, hx, stream, dev, reps=10):
     res = {}
     for name in ("gather", "sort"):
         total = 0.0
-        for _ in range(reps):
+        for it in range(reps + 1):                   # the first launch (module load, set-up) is not timed
             with torch.cuda.stream(stream):
                 flush.max()
                 i2, s2 = idx0.clone(), sc0.clone()
+                torch.cuda._sleep(_HOST_LEAD_CYCLES)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             if name == "gather":
@@ -296,7 +307,7 @@ def after_select_timings(api, hx, stream, dev, reps=10):
                 api.dsa_sort_selection(i2, s2, stream=stream)
             e1.record(stream)
             stream.synchronize()
-            total += e0.elapsed_time(e1)
+            total += e0.elapsed_time(e1) if it else 0.0
         res[name] = total / reps
     api.dsa_check_device_errors(stream)
     valid = int((idx0 >= 0).sum().item())
@@ -328,9 +339,10 @@ def rope_timings(api, stream, dev, reps=10):
     res = {}
     for name in ("queries", "keys"):
         total = 0.0
-        for _ in range(reps):
+        for it in range(reps + 1):                   # the first launch (module load, set-up) is not timed
             with torch.cuda.stream(stream):
                 flush.max()
+                torch.cuda._sleep(_HOST_LEAD_CYCLES)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             if name == "queries":
@@ -340,7 +352,7 @@ def rope_timings(api, stream, dev, reps=10):
                 api.dsa_indexer_kcache_append_rope(cache, k, rows, pos_k, rope_dim=64, interleaved=False, stream=stream)
             e1.record(stream)
             stream.synchronize()
-            total += e0.elapsed_time(e1)
+            total += e0.elapsed_time(e1) if it else 0.0
         res[name] = total / reps
     api.dsa_check_device_errors(stream)
     hbm = peaks()["hbm"]
@@ -378,6 +390,7 @@ def compressed_timings(api, hx, stream, dev, m=4, reps=10):
     for _ in range(reps):
         with torch.cuda.stream(stream):
             flush.max()
+            torch.cuda._sleep(_HOST_LEAD_CYCLES)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         call()
@@ -581,13 +594,20 @@ def run_ours(args):
     rows_h = hx.rows_host.pin_memory()
 
     # Each step uploads its inputs from pinned host memory and reads its selection back.
-    # Decode goes through the library's one-call host step (dsa_indexer_decode_host); prefill
+    # Decode goes through the library's one-call host step (dsa_indexer_decode_host with a
+    # completion event: the read-back of a step overlaps the kernels of the next); prefill
     # copies around the device call.  Steps are enqueued back to back (the host does not wait
-    # for each one); the events below bracket all of them on the stream.
+    # for each one); the events below bracket all of them, the end event placed after the
+    # last step's read-back has completed.
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    last = [None]
+
     def e2e_step():
         if hx.decode:
+            ev = done[0] if last[0] is not done[0] else done[1]
             api.dsa_indexer_decode_host(q_h, w_h, k_h, rows_h, hx.cache, hx.seq_lens, hx.q_lens, hx.wl.top_k,
-                                        oi_h, os_h, k_base=hx.k_base, stream=stream)
+                                        oi_h, os_h, k_base=hx.k_base, stream=stream, done_event=ev)
+            last[0] = ev
             return
         with torch.cuda.stream(stream):
             k_d.copy_(k_h, non_blocking=True)
@@ -599,15 +619,18 @@ def run_ours(args):
 
     for _ in range(3):
         e2e_step()
-    stream.synchronize()
+    torch.cuda.synchronize(dev)
     E = max(1, args.e2e_steps if hx.decode else min(args.e2e_steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
+    stream.synchronize()                     # the first upload (on the library's copy stream) starts after e0
     for _ in range(E):
         e2e_step()
+    if last[0] is not None:
+        stream.wait_event(last[0])           # every read-back has completed (one copy stream, in order)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, dist if world > 1 else None)
@@ -677,10 +700,23 @@ def run_ours(args):
     return 0
 
 
+def run_only(args):
+    import torch
+
+    from sparse_attention_token_02_b200 import api
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    if args.only == "rope":
+        print(json.dumps({"rope_fused": rope_timings(api, stream, dev, reps=args.reps)}), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only:
+        return run_only(args)
     return run_ours(args)
 
 

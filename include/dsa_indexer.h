@@ -169,16 +169,33 @@ DSA_API dsa_status_t dsa_indexer_decode(const dsa_query_t* q, const dsa_kcache_t
  *   3. copies the selection back into out_idx_host / out_score_host [T, top_k].
  * Here q->data and q->scale are HOST pointers, like every *_host argument.  Page-locked
  * host memory keeps the copies asynchronous; pageable memory works, with CUDA staging it.
- * The device copies live in library-owned buffers of `stream`, reused by the next call on
- * that stream (stream order makes this safe); the host outputs are complete once the
- * stream has finished (e.g. dsa_check_device_errors).  n_new may be 0.  Not capturable in
- * a CUDA graph (DSA_ERR_UNSUPPORTED while `stream` is capturing).
+ * The copies run on two copy streams of the library (one per direction) and the device
+ * copies live in two library-owned slots of `stream` used in turn, so the uploads of one
+ * call overlap the kernels of the previous one; events order everything against `stream`.
+ * The host inputs must stay unchanged, and the host outputs are complete, once `stream`
+ * has finished (e.g. dsa_check_device_errors).  n_new may be 0.  Not capturable in a CUDA
+ * graph (DSA_ERR_UNSUPPORTED while `stream` is capturing).
  */
 DSA_API dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
                                              const void* k_new_host, dsa_dtype_t k_new_dtype,
                                              const int64_t* dst_rows_host, int32_t n_new, const dsa_batch_t* batch,
                                              int32_t top_k, int32_t* out_idx_host, float* out_score_host,
                                              void* stream);
+
+/*
+ * dsa_indexer_decode_host without the read-back on `stream`: the device-to-host copies of
+ * the selection are ordered only on the library's copy stream, and done_event (a
+ * cudaEvent_t the caller created, required) is recorded there once out_idx_host and
+ * out_score_host are complete; wait on it (cudaEventSynchronize, cudaStreamWaitEvent)
+ * before reading them.  `stream` does not wait for the read-back, so the read-back of one
+ * step overlaps the kernels of the next.  Two calls in flight use the two slots: a third
+ * call waits on the device for the first one's read-back before reusing its slot.
+ */
+DSA_API dsa_status_t dsa_indexer_decode_host_async(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                                   const void* k_new_host, dsa_dtype_t k_new_dtype,
+                                                   const int64_t* dst_rows_host, int32_t n_new,
+                                                   const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
+                                                   float* out_score_host, void* stream, void* done_event);
 
 /*
  * The scores alone, without selection (the first page's index_scores, §3):
@@ -245,7 +262,8 @@ DSA_API dsa_status_t dsa_indexer_decode_compressed(const dsa_query_t* q, const d
 typedef struct {
   int32_t rope_dim;     /* leading values that rotate: even, <= d_I (0: none)               */
   int32_t interleaved;  /* 1: pairs (2i, 2i+1); 0: pairs (i, i + rope_dim/2), which needs     */
-                        /*    rope_dim / 2 = 2^m * d_I / 32 (e.g. d_I = 128: 8, 16, 32, 64, 128)   */
+                        /*    rope_dim / 2 = 2^m * d_I / 32 and a multiple of 8                 */
+                        /*    (d_I = 128: rope_dim 16, 32, 64, 128; d_I = 64: 16, 32, 64)       */
   double base;          /* 10000 in the published form                                        */
 } dsa_rope_t;
 
@@ -262,7 +280,9 @@ DSA_API dsa_status_t dsa_indexer_kcache_append_rope(const dsa_kcache_t* kc, cons
  * Queries q_src [T, H_I, d_I] (bf16 or fp32, pre-RoPE, device): every head of token t is
  * rotated at positions[t] (device int32 [T]) and written to q_dst [T, H_I, d_I] as bf16
  * (dst_dtype DSA_BF16) or as E4M3 codes with one scale per token in q_scale [T]
- * (DSA_FP8_E4M3, as dsa_quantize_rows_fp8).  H_I <= 128, d_I 64 or 128.
+ * (DSA_FP8_E4M3, as dsa_quantize_rows_fp8).  H_I <= 128, d_I 64 or 128; q_src and q_dst
+ * 16-byte aligned (DSA_ERR_INVALID_ARG otherwise).  A timed-out copy wait inside the kernel
+ * is reported by dsa_check_device_errors.
  */
 DSA_API dsa_status_t dsa_rope_queries(const void* q_src, dsa_dtype_t src_dtype, int64_t T, int32_t H_I, int32_t d_I,
                                       const int32_t* positions, const dsa_rope_t* rope, void* q_dst,

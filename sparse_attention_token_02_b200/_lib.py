@@ -25,6 +25,7 @@ EXPORTED = (
     "dsa_indexer_decode",
     "dsa_indexer_decode_noalloc",
     "dsa_indexer_decode_host",
+    "dsa_indexer_decode_host_async",
     "dsa_indexer_decode_compressed",
     "dsa_indexer_kcache_append_rope",
     "dsa_rope_queries",
@@ -94,6 +95,9 @@ def load() -> ctypes.CDLL:
     lib.dsa_indexer_decode_noalloc.restype = st
     lib.dsa_indexer_decode_host.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V, V]
     lib.dsa_indexer_decode_host.restype = st
+    lib.dsa_indexer_decode_host_async.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V,
+                                                  V, V]
+    lib.dsa_indexer_decode_host_async.restype = st
     lib.dsa_indexer_decode_compressed.argtypes = [P(Query), P(KCache), V, P(Batch), I32, I32, V, V, V]
     lib.dsa_indexer_decode_compressed.restype = st
     lib.dsa_indexer_kcache_append_rope.argtypes = [P(KCache), V, ctypes.c_int, V, V, I32, P(Rope), V]

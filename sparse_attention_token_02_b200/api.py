@@ -170,13 +170,16 @@ def dsa_indexer_decode_noalloc(q, cache: IndexerKCache, w, seq_lens, q_lens, top
 
 
 def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: IndexerKCache, seq_lens, q_lens,
-                            top_k, out_idx_host, out_score_host, q_scale_host=None, k_base=None, stream=None):
+                            top_k, out_idx_host, out_score_host, q_scale_host=None, k_base=None, stream=None,
+                            done_event=None):
     """One decode step from HOST tensors in a single library call (dsa_indexer_decode_host):
     upload the new keys (bf16 or fp32 [n_new, d_I], cache rows ``dst_rows_host`` int64), queries
     [T, H_I, d_I] (bf16, or uint8 E4M3 codes with ``q_scale_host``) and weights [T, H_I] fp32,
     append, score + select, and copy the selection into ``out_idx_host`` int32 / ``out_score_host``
-    fp32 [T, top_k].  Returns at once; the host outputs are complete when ``stream`` has finished.
-    Pinned host tensors keep the copies asynchronous."""
+    fp32 [T, top_k].  Returns at once; the host outputs are complete when ``stream`` has finished,
+    or, with ``done_event`` (a torch.cuda.Event; dsa_indexer_decode_host_async), once that event
+    has completed, while ``stream`` goes on without waiting for the read-back.  Pinned host
+    tensors keep the copies asynchronous."""
     for t in (q_host, w_host, k_new_host, dst_rows_host, out_idx_host, out_score_host, q_scale_host):
         if t is not None and (t.is_cuda or not t.is_contiguous()):
             raise ValueError("dsa_indexer_decode_host takes contiguous host tensors")
@@ -191,10 +194,15 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
                q_host.shape[1], q_host.shape[2])
     kc = cache.c()
     n_new = int(k_new_host.shape[0]) if k_new_host is not None else 0
-    check(_lib.load().dsa_indexer_decode_host(ctypes.byref(qq), ctypes.byref(kc), _ptr(w_host), _ptr(k_new_host),
-                                              _dtype_code(k_new_host) if n_new else DSA_BF16, _ptr(dst_rows_host),
-                                              n_new, ctypes.byref(b.c), top_k, _ptr(out_idx_host),
-                                              _ptr(out_score_host), _stream(stream)))
+    args = (ctypes.byref(qq), ctypes.byref(kc), _ptr(w_host), _ptr(k_new_host),
+            _dtype_code(k_new_host) if n_new else DSA_BF16, _ptr(dst_rows_host), n_new, ctypes.byref(b.c), top_k,
+            _ptr(out_idx_host), _ptr(out_score_host), _stream(stream))
+    if done_event is None:
+        check(_lib.load().dsa_indexer_decode_host(*args))
+        return
+    if not done_event.cuda_event:               # torch creates its events on their first record
+        done_event.record(torch.cuda.current_stream() if stream is None else stream)
+    check(_lib.load().dsa_indexer_decode_host_async(*args, ctypes.c_void_p(done_event.cuda_event)))
 
 
 def dsa_selftest_wait_expiry(limit_cycles=100000, stream=None):

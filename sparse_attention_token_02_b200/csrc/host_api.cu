@@ -140,8 +140,20 @@ struct Ctx {
   MetaLayout layout;
   void* cur_meta = nullptr;       // tables of the cached plan
   float* cur_scores = nullptr;    // score workspace of the cached plan
-  void* d_host_stage = nullptr;   // dsa_indexer_decode_host: device copies of the step's inputs/outputs
-  size_t host_stage_cap = 0;
+  // dsa_indexer_decode_host: device copies of a step's inputs and outputs, in two slots used in
+  // turn, filled and read back on the context's own copy streams so that the copies of one
+  // step overlap the compute of its neighbours
+  struct StepSlot {
+    void* d = nullptr;
+    size_t cap = 0;
+    cudaEvent_t in_done = nullptr;    // the inputs have landed
+    cudaEvent_t computed = nullptr;   // the step's kernels are done with the slot's inputs and outputs
+    cudaEvent_t out_done = nullptr;   // the outputs have been copied to the host
+    bool used = false;
+  };
+  StepSlot step[2];
+  int step_next = 0;
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
 };
 
 std::mutex g_mu;
@@ -819,10 +831,30 @@ dsa_status_t dsa_indexer_decode(const dsa_query_t* q, const dsa_kcache_t* kc, co
   return run_indexer(Mode::Decode, q, kc, w, batch, top_k, out_idx, out_score, nullptr, 0, stream);
 }
 
-dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
-                                     const void* k_new_host, dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host,
-                                     int32_t n_new, const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
-                                     float* out_score_host, void* stream_v) {
+// Copy streams and slot events of the host step, created on first use.
+static dsa_status_t ensure_step_streams(Ctx* c) {
+  if (c->copy_in) return DSA_OK;
+  DSA_CUDA_TRY(cudaStreamCreateWithFlags(&c->copy_in, cudaStreamNonBlocking), "cudaStreamCreate(copy in)");
+  DSA_CUDA_TRY(cudaStreamCreateWithFlags(&c->copy_out, cudaStreamNonBlocking), "cudaStreamCreate(copy out)");
+  for (auto& sl : c->step) {
+    DSA_CUDA_TRY(cudaEventCreateWithFlags(&sl.in_done, cudaEventDisableTiming), "cudaEventCreate");
+    DSA_CUDA_TRY(cudaEventCreateWithFlags(&sl.computed, cudaEventDisableTiming), "cudaEventCreate");
+    DSA_CUDA_TRY(cudaEventCreateWithFlags(&sl.out_done, cudaEventDisableTiming), "cudaEventCreate");
+  }
+  return DSA_OK;
+}
+
+// The host step.  Slot i % 2 holds step i's inputs and outputs:
+//   copy_in : [wait computed(i-2)] H2D inputs            [record in_done(i)]
+//   stream  : [wait in_done(i), out_done(i-2)] append, quantise, decode   [record computed(i)]
+//   copy_out: [wait computed(i)] D2H outputs             [record out_done(i), done_event]
+// With join, `stream` then waits for out_done(i), so the host outputs are complete when the
+// stream is (the uploads of the next call still overlap this call's compute); without, the
+// caller waits on done_event.
+static dsa_status_t decode_host_step(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host, const void* k_new_host,
+                              dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host, int32_t n_new,
+                              const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host, float* out_score_host,
+                              void* stream_v, cudaEvent_t done_event, bool join) {
   g_last_error.clear();
   dsa_status_t st = check_cache(kc);
   if (st != DSA_OK) return st;
@@ -846,8 +878,9 @@ dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* k
   if (cap != cudaStreamCaptureStatusNone) return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_decode_host cannot be captured");
   Ctx* c = nullptr;
   if ((st = get_ctx(stream, &c)) != DSA_OK) return st;
+  if ((st = ensure_step_streams(c)) != DSA_OK) return st;
 
-  // device staging: [k_new | dst_rows | q | q_scale | w | out_idx | out_score | q8 | q8_scale],
+  // slot layout: [k_new | dst_rows | q | q_scale | w | out_idx | out_score | q8 | q8_scale],
   // 256-byte aligned parts (the last two only when bf16 queries meet an FP8 cache)
   const size_t esz_k = k_new_dtype == DSA_F32 ? 4 : 2, esz_q = q->dtype == DSA_FP8_E4M3 ? 1 : 2;
   const size_t q_elems = size_t(T) * q->H_I * q->d_I;
@@ -858,25 +891,32 @@ dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* k
   const size_t o_w = o_qs + align_up(b_qs), o_oi = o_w + align_up(b_w), o_os = o_oi + align_up(b_out);
   const size_t o_q8 = o_os + align_up(b_out), o_q8s = o_q8 + (quantise_q ? align_up(q_elems) : 0);
   const size_t total = o_q8s + (quantise_q ? align_up(size_t(T) * 4) : 0);
-  if (total > c->host_stage_cap) {
-    if (c->d_host_stage) {
-      DSA_CUDA_TRY(cudaStreamSynchronize(stream), "cudaStreamSynchronize");   // earlier calls may still read it
-      DSA_CUDA_TRY(cudaFree(c->d_host_stage), "cudaFree");
-      c->d_host_stage = nullptr;
-      c->host_stage_cap = 0;
+  Ctx::StepSlot& sl = c->step[c->step_next];
+  if (total > sl.cap) {
+    if (sl.d) {
+      DSA_CUDA_TRY(cudaEventSynchronize(sl.out_done), "cudaEventSynchronize");   // its last step is over
+      DSA_CUDA_TRY(cudaFree(sl.d), "cudaFree");
+      sl.d = nullptr;
+      sl.cap = 0;
     }
-    DSA_CUDA_TRY(cudaMalloc(&c->d_host_stage, total), "cudaMalloc(host-step staging)");
-    c->host_stage_cap = total;
+    DSA_CUDA_TRY(cudaMalloc(&sl.d, total), "cudaMalloc(host-step staging)");
+    sl.cap = total;
   }
-  char* d = static_cast<char*>(c->d_host_stage);
+  char* d = static_cast<char*>(sl.d);
+  if (sl.used) DSA_CUDA_TRY(cudaStreamWaitEvent(c->copy_in, sl.computed, 0), "cudaStreamWaitEvent");
   auto h2d = [&](size_t off, const void* src, size_t bytes) -> cudaError_t {
-    return bytes ? cudaMemcpyAsync(d + off, src, bytes, cudaMemcpyHostToDevice, stream) : cudaSuccess;
+    return bytes ? cudaMemcpyAsync(d + off, src, bytes, cudaMemcpyHostToDevice, c->copy_in) : cudaSuccess;
   };
   DSA_CUDA_TRY(h2d(0, k_new_host, b_k), "cudaMemcpyAsync(k_new)");
   DSA_CUDA_TRY(h2d(o_rows, dst_rows_host, b_rows), "cudaMemcpyAsync(dst_rows)");
   DSA_CUDA_TRY(h2d(o_q, q->data, b_q), "cudaMemcpyAsync(q)");
   DSA_CUDA_TRY(h2d(o_qs, q->scale, b_qs), "cudaMemcpyAsync(q_scale)");
   DSA_CUDA_TRY(h2d(o_w, w_host, b_w), "cudaMemcpyAsync(w)");
+  DSA_CUDA_TRY(cudaEventRecord(sl.in_done, c->copy_in), "cudaEventRecord");
+  DSA_CUDA_TRY(cudaStreamWaitEvent(stream, sl.in_done, 0), "cudaStreamWaitEvent");
+  if (sl.used) DSA_CUDA_TRY(cudaStreamWaitEvent(stream, sl.out_done, 0), "cudaStreamWaitEvent");
+  sl.used = true;
+  c->step_next ^= 1;
   if (n_new > 0 &&
       (st = dsa_indexer_kcache_append(kc, d, k_new_dtype, reinterpret_cast<const int64_t*>(d + o_rows), n_new,
                                       stream_v)) != DSA_OK)
@@ -897,11 +937,38 @@ dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* k
   if ((st = dsa_indexer_decode(&qd, kc, reinterpret_cast<const float*>(d + o_w), batch, top_k, oi, os, stream_v)) !=
       DSA_OK)
     return st;
+  DSA_CUDA_TRY(cudaEventRecord(sl.computed, stream), "cudaEventRecord");
+  DSA_CUDA_TRY(cudaStreamWaitEvent(c->copy_out, sl.computed, 0), "cudaStreamWaitEvent");
   if (b_out) {
-    DSA_CUDA_TRY(cudaMemcpyAsync(out_idx_host, oi, b_out, cudaMemcpyDeviceToHost, stream), "cudaMemcpyAsync(out_idx)");
-    DSA_CUDA_TRY(cudaMemcpyAsync(out_score_host, os, b_out, cudaMemcpyDeviceToHost, stream), "cudaMemcpyAsync(out_score)");
+    DSA_CUDA_TRY(cudaMemcpyAsync(out_idx_host, oi, b_out, cudaMemcpyDeviceToHost, c->copy_out), "cudaMemcpyAsync(out_idx)");
+    DSA_CUDA_TRY(cudaMemcpyAsync(out_score_host, os, b_out, cudaMemcpyDeviceToHost, c->copy_out),
+                 "cudaMemcpyAsync(out_score)");
   }
+  DSA_CUDA_TRY(cudaEventRecord(sl.out_done, c->copy_out), "cudaEventRecord");
+  if (done_event) DSA_CUDA_TRY(cudaEventRecord(done_event, c->copy_out), "cudaEventRecord(done_event)");
+  if (join) DSA_CUDA_TRY(cudaStreamWaitEvent(stream, sl.out_done, 0), "cudaStreamWaitEvent");
   return DSA_OK;
+}
+
+dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                     const void* k_new_host, dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host,
+                                     int32_t n_new, const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
+                                     float* out_score_host, void* stream_v) {
+  return decode_host_step(q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
+                          out_score_host, stream_v, nullptr, true);
+}
+
+dsa_status_t dsa_indexer_decode_host_async(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                           const void* k_new_host, dsa_dtype_t k_new_dtype,
+                                           const int64_t* dst_rows_host, int32_t n_new, const dsa_batch_t* batch,
+                                           int32_t top_k, int32_t* out_idx_host, float* out_score_host,
+                                           void* stream_v, void* done_event) {
+  if (!done_event) {
+    g_last_error.clear();
+    return fail(DSA_ERR_INVALID_ARG, "done_event is NULL");
+  }
+  return decode_host_step(q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
+                          out_score_host, stream_v, static_cast<cudaEvent_t>(done_event), false);
 }
 
 dsa_status_t dsa_indexer_decode_compressed(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
@@ -1004,12 +1071,15 @@ dsa_status_t dsa_rope_queries(const void* q_src, dsa_dtype_t src_dtype, int64_t 
   if (T > 0x7FFFFFFF) return fail(DSA_ERR_UNSUPPORTED, "too many tokens for one launch");
   const RopeParams rp = rope_params(*rope);
   if (!rope_shape_supported(d, H, rp)) return fail(DSA_ERR_UNSUPPORTED, "unsupported RoPE shape (H_I %d, d_I %d)", H, d);
+  if (reinterpret_cast<uintptr_t>(q_src) % 16 || reinterpret_cast<uintptr_t>(q_dst) % 16)
+    return fail(DSA_ERR_INVALID_ARG, "q_src and q_dst must be 16-byte aligned");
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
   Ctx* c = nullptr;
   dsa_status_t st = get_ctx(stream, &c);
   if (st != DSA_OK) return st;
+  if (!g_sms) g_sms = num_sms(c->device);
   DSA_CUDA_TRY(launch_rope_queries(q_src, src_dtype == DSA_F32, T, H, d, positions, rp, dst_dtype == DSA_FP8_E4M3,
-                                   q_dst, q_scale, stream),
+                                   q_dst, q_scale, c->d_err, g_sms, stream),
                "RoPE query kernel launch");
   ++g_launches;
   return DSA_OK;

@@ -131,7 +131,7 @@ cudaError_t launch_rope_append(const void* src, int src_is_f32, int64_t rows, in
                                float* scale, int* err, cudaStream_t stream);
 cudaError_t launch_rope_queries(const void* src, int src_is_f32, int64_t T, int32_t H, int32_t d,
                                 const int32_t* positions, const RopeParams& r, int fp8, void* dst, float* scale,
-                                cudaStream_t stream);
+                                int* err, int sms, cudaStream_t stream);
 
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
 cudaError_t launch_wait_expiry(long long limit_cycles, int* err, cudaStream_t stream);

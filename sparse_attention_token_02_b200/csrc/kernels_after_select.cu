@@ -24,54 +24,66 @@ constexpr int kGatherThreads = 256;
 constexpr int kMaxRowVecs = 32 * 8;           // rows up to 4 KB: at most 8 vectors per lane
 constexpr int kGatherInFlight = 8;            // 16-byte loads per lane issued together
 
-// One warp copies RPW rows per iteration, VPL vectors per lane per row (VPL * 32 >= the
-// row's vectors), all RPW * VPL loads of the iteration in flight before any store.
+constexpr int kGatherCtasPerSm = 4;           // resident CTAs per SM the grid is sized for
+
+// Source row of output entry o: -2 none (past the end), -1 a padding entry (a zero row),
+// else the row of src.  An out-of-range row is reported and written as zeros.
+__device__ __forceinline__ int64_t gather_src_row(const int32_t* __restrict__ idx, const int64_t* __restrict__ row_base,
+                                                  int64_t o, int64_t end, int32_t top_k, int64_t src_rows, int* err) {
+  if (o >= end) return -2;
+  const int32_t i = idx[o];
+  if (i < 0) return -1;
+  const int64_t sr = row_base[o / top_k] + i;
+  if (sr < 0 || sr >= src_rows) {
+    record_error(err, DSA_DEVERR_BOUNDS, static_cast<int>(o / top_k));
+    return -1;
+  }
+  return sr;
+}
+
+// Warp w copies the contiguous output entries [n_out * w / W, n_out * (w + 1) / W) (W warps
+// in the grid, so the share of every warp is the same to within one row).  It resolves the
+// source rows of up to 32 entries at once (one entry per lane, so the index and row-base
+// loads of a batch overlap), then copies them RPW rows at a time, VPL 16-byte vectors per
+// lane per row (VPL * 32 >= the row's vectors), all RPW * VPL loads in flight before any store.
 template <int VPL, int RPW>
-__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4* __restrict__ src, int64_t src_rows,
-                                                                     int32_t row_vecs, const int32_t* __restrict__ idx,
-                                                                     const int64_t* __restrict__ row_base,
-                                                                     int64_t n_out, int32_t top_k,
-                                                                     uint4* __restrict__ dst, int* err) {
+__global__ void __launch_bounds__(kGatherThreads, kGatherCtasPerSm)
+gather_rows_kernel(const uint4* __restrict__ src, int64_t src_rows, int32_t row_vecs, const int32_t* __restrict__ idx,
+                   const int64_t* __restrict__ row_base, int64_t n_out, int32_t top_k, uint4* __restrict__ dst,
+                   int* err) {
   static_assert(VPL * RPW == kGatherInFlight, "loads in flight per lane");
   grid_dependency_wait();                     // the selection comes from the previous kernel
   const int lane = threadIdx.x & 31;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kGatherThreads + threadIdx.x) >> 5;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kGatherThreads + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kGatherThreads) >> 5;
-  for (int64_t o0 = warp0 * RPW; o0 < n_out; o0 += n_warps * RPW) {
-    int64_t srow[RPW];
+  const int64_t begin = n_out * warp / n_warps, end = n_out * (warp + 1) / n_warps;
+  for (int64_t b0 = begin; b0 < end; b0 += 32) {
+    const int64_t mine = gather_src_row(idx, row_base, b0 + lane, end, top_k, src_rows, err);
+    const int batch = end - b0 < 32 ? static_cast<int>(end - b0) : 32;
+    for (int g = 0; g < batch; g += RPW) {
+      int64_t srow[RPW];
 #pragma unroll
-    for (int q = 0; q < RPW; ++q) {
-      const int64_t o = o0 + q;
-      srow[q] = -2;                                       // -2: no such output row
-      if (o < n_out) {
-        const int32_t i = idx[o];
-        srow[q] = -1;
-        if (i >= 0) {
-          const int64_t sr = row_base[o / top_k] + i;
-          if (sr < 0 || sr >= src_rows) {
-            if (lane == 0) record_error(err, DSA_DEVERR_BOUNDS, static_cast<int>(o / top_k));
-          } else {
-            srow[q] = sr;
-          }
+      for (int q = 0; q < RPW; ++q) srow[q] = __shfl_sync(0xffffffffu, mine, (g + q) & 31);
+#pragma unroll
+      for (int q = 0; q < RPW; ++q)
+        if (g + q >= batch) srow[q] = -2;
+      uint4 v[RPW][VPL];
+#pragma unroll
+      for (int q = 0; q < RPW; ++q)
+#pragma unroll
+        for (int u = 0; u < VPL; ++u) {
+          const int c = u * 32 + lane;
+          v[q][u] = make_uint4(0u, 0u, 0u, 0u);
+          if (srow[q] >= 0 && c < row_vecs) v[q][u] = __ldcs(src + srow[q] * row_vecs + c);
         }
-      }
+#pragma unroll
+      for (int q = 0; q < RPW; ++q)
+#pragma unroll
+        for (int u = 0; u < VPL; ++u) {
+          const int c = u * 32 + lane;
+          if (srow[q] != -2 && c < row_vecs) __stcs(dst + (b0 + g + q) * row_vecs + c, v[q][u]);
+        }
     }
-    uint4 v[RPW][VPL];
-#pragma unroll
-    for (int q = 0; q < RPW; ++q)
-#pragma unroll
-      for (int u = 0; u < VPL; ++u) {
-        const int c = u * 32 + lane;
-        v[q][u] = make_uint4(0u, 0u, 0u, 0u);
-        if (srow[q] >= 0 && c < row_vecs) v[q][u] = __ldcs(src + srow[q] * row_vecs + c);
-      }
-#pragma unroll
-    for (int q = 0; q < RPW; ++q)
-#pragma unroll
-      for (int u = 0; u < VPL; ++u) {
-        const int c = u * 32 + lane;
-        if (srow[q] != -2 && c < row_vecs) __stcs(dst + (o0 + q) * row_vecs + c, v[q][u]);
-      }
   }
 }
 
@@ -208,7 +220,7 @@ cudaError_t launch_gather_rows(const void* src, int64_t src_rows, int32_t row_by
   const int vpl = row_vecs <= 32 ? 1 : row_vecs <= 64 ? 2 : row_vecs <= 128 ? 4 : 8;
   const int rpw = kGatherInFlight / vpl;
   const int64_t want = (n_out + rpw * (kGatherThreads / 32) - 1) / (rpw * (kGatherThreads / 32));
-  const int64_t cap = static_cast<int64_t>(sms) * 4;     // one resident wave (about 64 registers a thread)
+  const int64_t cap = static_cast<int64_t>(sms) * kGatherCtasPerSm;   // one resident wave
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(want < cap ? want : cap)), dim3(kGatherThreads),
                                       stream, attr);

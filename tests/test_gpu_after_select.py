@@ -48,6 +48,22 @@ def test_gather_rows_bit_exact(selection, row_bytes):
     assert np.array_equal(out.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("rows,row_bytes", [(300, 16), (40, 1024), (16, 4096), (7, 48)])
+def test_gather_rows_many_batches_per_warp(rows, row_bytes):
+    # synthetic selections (padding included) large enough that every warp copies several
+    # 32-entry batches, over the narrowest, the widest and an odd number of vectors per row
+    top_k, src_rows = 2048, 50000
+    rng = np.random.default_rng(rows * row_bytes)
+    idx = rng.integers(0, 40000, (rows, top_k)).astype(np.int32)
+    idx[rng.random((rows, top_k)) < 0.1] = -1
+    base = rng.integers(0, src_rows - 40000, rows).astype(np.int64)
+    src = torch.randint(0, 256, (src_rows, row_bytes), dtype=torch.uint8,
+                        generator=torch.Generator().manual_seed(rows)).cuda()
+    out = api.dsa_gather_rows(src, torch.from_numpy(idx).cuda(), torch.from_numpy(base).cuda())
+    api.dsa_check_device_errors()
+    assert np.array_equal(out.cpu().numpy(), A.gather_rows(src.cpu().numpy(), idx, base))
+
+
 def test_gather_rows_bf16_view_and_out_of_range_row(selection):
     wl, idx, _, base = selection
     rows = int(sum(wl.seq_lens))

@@ -391,6 +391,54 @@ def test_decode_host_step_equals_device_calls_two_calls_in_a_row(name):
             np.testing.assert_array_equal(gs, rs)
 
 
+@pytest.mark.parametrize("name", ["bf16", "fp8"])
+def test_decode_host_step_async_three_calls_in_flight(name):
+    # three steps with different inputs and outputs enqueued without waiting (the third reuses
+    # the first one's slot), each read back under its own completion event
+    base = W.decode() if name == "bf16" else W.decode8()
+    L, q_lens = (4100, 700, 2049), (2, 1, 1)
+    wl = W.scaled(base, seq_lens=L, q_lens=q_lens, seed=90)
+    up = Uploaded(wl)
+    rows = np.concatenate([up.k_base[b] + np.arange(Lb - n, Lb) for b, (Lb, n) in enumerate(zip(L, q_lens))])
+    k_bits = np.concatenate(up.inp["k_bits"])[rows]
+    k_h = torch.from_numpy(np.ascontiguousarray(k_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    rows_h = torch.from_numpy(rows.astype(np.int64)).pin_memory()
+    s = torch.cuda.Stream()
+    steps = []
+    for call in range(3):
+        rng = np.random.default_rng(200 + call)
+        q_bits = W.f32_to_bf16_bits((rng.standard_normal(up.inp["q_bits"].shape) / 11.3).astype(np.float32))
+        w = W.softmax_rows(rng.standard_normal(up.inp["w"].shape).astype(np.float32))
+        q_h = torch.from_numpy(np.ascontiguousarray(q_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+        w_h = torch.from_numpy(w).pin_memory()
+        oi_h = torch.full((wl.total_q, wl.top_k), 7, dtype=torch.int32).pin_memory()
+        os_h = torch.zeros((wl.total_q, wl.top_k), dtype=torch.float32).pin_memory()
+        ev = torch.cuda.Event()
+        api.dsa_indexer_decode_host(q_h, w_h, k_h, rows_h, up.cache, L, q_lens, wl.top_k, oi_h, os_h,
+                                    k_base=up.k_base, stream=s, done_event=ev)
+        steps.append((q_h, w_h, oi_h, os_h, ev))
+    for q_h, w_h, oi_h, os_h, ev in steps:
+        ev.synchronize()
+        q_dev, q_scale = _device_q(up, q_h)
+        ref_i, ref_s = api.dsa_indexer_decode(q_dev, up.cache, w_h.cuda(), L, q_lens, wl.top_k, k_base=up.k_base,
+                                              q_scale=q_scale)
+        ref_i, ref_s = ref_i.cpu().numpy(), ref_s.cpu().numpy()
+        for (gi, gs), (ri, rs) in zip(_sorted_rows(oi_h.numpy(), os_h.numpy()), _sorted_rows(ref_i, ref_s)):
+            assert np.array_equal(gi, ri)
+            np.testing.assert_array_equal(gs, rs)
+    api.dsa_check_device_errors(s)
+
+
+def _device_q(up, q_h):
+    """The queries the device call takes for this cache: (bf16, None), or (E4M3 codes, scales)
+    quantised on the device as the host step does for an FP8 cache."""
+    q = q_h.cuda()
+    if not up.cache.fp8:
+        return q, None
+    codes, scale = api.dsa_quantize_rows_fp8(q.reshape(q.shape[0], -1))
+    return codes.reshape(q.shape), scale
+
+
 def test_decode_host_step_rejects_bad_arguments():
     wl = W.scaled(W.decode(), seq_lens=(300,), q_lens=(1,))
     up = Uploaded(wl)

@@ -108,6 +108,35 @@ def test_rope_queries_against_oracle(interleaved, rope_dim, fp8):
         _within_one_bf16_step(res, ref)
 
 
+@pytest.mark.parametrize("T,H,d,f32,fp8,interleaved,rope_dim", [
+    (4000, 64, 128, False, True, False, 64),     # several tokens per shared-memory slot
+    (10000, 8, 64, True, True, True, None),      # fp32 source, eight-slot rings
+    (700, 128, 128, False, False, True, 64),     # the largest token (eight chunks a thread)
+    (301, 3, 64, True, False, False, 32),        # heads not a multiple of the warps
+])
+def test_rope_queries_ring_shapes(T, H, d, f32, fp8, interleaved, rope_dim):
+    rng = np.random.default_rng(T + H)
+    x = rng.standard_normal((T, H, d)).astype(np.float32)
+    if f32:
+        src, ref_in = torch.from_numpy(x).cuda(), x.astype(np.float64)
+    else:
+        bits = W.f32_to_bf16_bits(x)
+        src = bits_to_bf16_tensor(bits, "cuda")
+        ref_in = F.bf16_bits_to_f64(bits.reshape(T * H, d)).reshape(T, H, d)
+    pos = rng.integers(0, 200000, T).astype(np.int32)
+    res = api.dsa_rope_queries(src, torch.from_numpy(pos).cuda(), fp8=fp8, rope_dim=rope_dim, interleaved=interleaved)
+    api.dsa_check_device_errors()
+    ref = R.rope_heads(ref_in, pos, rope_dim or d, interleaved=interleaved)
+    if fp8:
+        codes, scale = res
+        np.testing.assert_allclose(scale.cpu().numpy(),
+                                   np.abs(ref).reshape(T, -1).max(axis=1).astype(np.float32) / np.float32(448),
+                                   rtol=1e-6)
+        _within_one_e4m3_step(codes, scale, ref)
+    else:
+        _within_one_bf16_step(res, ref)
+
+
 def test_rope_rejects_unsupported_layouts():
     cache = api.IndexerKCache.empty(8, 128, False)
     k = torch.zeros(2, 128, dtype=torch.bfloat16, device="cuda")
