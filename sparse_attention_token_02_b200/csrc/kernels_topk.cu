@@ -6,7 +6,9 @@
 //   * one cluster of `cs` CTAs per row (distributed shared memory joins them); each
 //     thread loads EPT scores of its CTA's slice with 16-byte loads and maps each to
 //     an order-preserving uint32 key (larger float -> larger key);
-//   * the cluster reduces min and max key -> candidate key interval [lo, hi];
+//   * the cluster reduces min and max key -> candidate key interval [lo, hi]; when the
+//     logits epilogue has binned the row (decode), its coarse histogram gives the
+//     threshold bin directly and this level and the next are skipped;
 //   * refinement level: bin = (key - lo) >> shift, with shift chosen so the interval
 //     spans at most 2048 bins.  Histograms are built with shared atomics and summed
 //     into rank 0 over DSMEM; rank 0 finds the bin holding the k-th largest key,
@@ -106,6 +108,19 @@ __device__ __forceinline__ void find_threshold_bin(const uint32_t (&cnt)[PER], u
       *found_cnt = cnt[j];
     }
     above += cnt[j];
+  }
+}
+
+// PER consecutive bins starting at h, returned in descending bin order.
+template <int PER>
+__device__ __forceinline__ void load_bins_desc(const uint32_t* h, uint32_t (&c)[PER]) {
+#pragma unroll
+  for (int q = 0; q < PER / 4; ++q) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(h + 4 * q));
+    c[PER - 1 - 4 * q] = v.x;
+    c[PER - 2 - 4 * q] = v.y;
+    c[PER - 3 - 4 * q] = v.z;
+    c[PER - 4 - 4 * q] = v.w;
   }
 }
 
@@ -256,6 +271,12 @@ topk_kernel(const TopkArgs a) {
   __syncthreads();
   grid_dependency_wait();                     // the scores come from the previous kernel
 
+  // ---- the row's coarse histogram, when the logits epilogue built one (decode)
+  constexpr int kPer0 = kHistBins / kThreads;
+  uint32_t c0[kPer0];
+  if (a.row_hist)
+    load_bins_desc<kPer0>(a.row_hist + static_cast<int64_t>(row) * kHistBins + (kHistBins - kPer0 * (tid + 1)), c0);
+
   // ---- load the slice into registers as order-preserving keys (0 = absent)
   uint32_t key[EPT];
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
@@ -276,60 +297,72 @@ topk_kernel(const TopkArgs a) {
     }
   }
 
-  // ---- data-driven first level: bins spread over the row's key range
+  uint32_t bin_lo, bin_hi;
+  if (a.row_hist) {
+    // the histogram fixes the threshold bin B (every CTA of the cluster reads the same one)
+    find_threshold_bin<kPer0>(c0, kHistBins - 1 - kPer0 * tid, k, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt);
+    __syncthreads();
+    bin_lo = lvl_bin << kHistShift;
+    bin_hi = bin_lo | ((1u << kHistShift) - 1u);
+  } else {
+    // ---- data-driven first level: bins spread over the row's key range
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) {
-    atomicMin(&loc_min, kmin);
-    atomicMax(&loc_max, kmax);
-  }
-  cluster.sync();                             // every CTA's key range is published
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  {
-    uint32_t rmin[kMaxCluster], rmax[kMaxCluster];   // all remote loads in flight together
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      rmin[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_min, r) : 0xFFFFFFFFu;
-      rmax[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_max, r) : 0u;
+    for (int o = 16; o > 0; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
     }
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      lo = min(lo, rmin[r]);
-      hi = max(hi, rmax[r]);
+    if (lane == 0) {
+      atomicMin(&loc_min, kmin);
+      atomicMax(&loc_max, kmax);
     }
-  }
-  const int bits0 = hi > lo ? 32 - __clz(hi - lo) : 0;
-  const int shift0 = bits0 > 11 ? bits0 - 11 : 0;
+    cluster.sync();                           // every CTA's key range is published
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    {
+      uint32_t rmin[kMaxCluster], rmax[kMaxCluster];   // all remote loads in flight together
 #pragma unroll
-  for (int e = 0; e < EPT; ++e)
-    if (key[e]) atomicAdd(&hist[(key[e] - lo) >> shift0], 1u);
-  cluster.sync();                             // every CTA's histogram is complete
-  {
-    // every CTA sums the cluster's histograms and finds the bin of the k-th key
-    uint32_t c[kBinsPerThread];
+      for (int r = 0; r < kMaxCluster; ++r) {
+        rmin[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_min, r) : 0xFFFFFFFFu;
+        rmax[r] = r < static_cast<int>(cs) ? *cluster.map_shared_rank(&loc_max, r) : 0u;
+      }
 #pragma unroll
-    for (int j = 0; j < kBinsPerThread; ++j) c[j] = 0u;
-    // this thread's kBinsPerThread consecutive bins as one 16-byte load per rank, all in flight
-    const int b0 = kBins - (tid + 1) * kBinsPerThread;
-    uint4 part[kMaxCluster];
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r)
-      part[r] = r < static_cast<int>(cs) ? *reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, r) + b0)
-                                         : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      c[0] += part[r].w;       // bins in descending order: b0+3, b0+2, b0+1, b0
-      c[1] += part[r].z;
-      c[2] += part[r].y;
-      c[3] += part[r].x;
+      for (int r = 0; r < kMaxCluster; ++r) {
+        lo = min(lo, rmin[r]);
+        hi = max(hi, rmax[r]);
+      }
     }
-    find_threshold_bin<kBinsPerThread>(c, kBins - 1 - tid * kBinsPerThread, k, warp_sums, &lvl_bin, &lvl_above,
-                                       &lvl_cnt);
+    const int bits0 = hi > lo ? 32 - __clz(hi - lo) : 0;
+    const int shift0 = bits0 > 11 ? bits0 - 11 : 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e)
+      if (key[e]) atomicAdd(&hist[(key[e] - lo) >> shift0], 1u);
+    cluster.sync();                           // every CTA's histogram is complete
+    {
+      // every CTA sums the cluster's histograms and finds the bin of the k-th key
+      uint32_t c[kBinsPerThread];
+#pragma unroll
+      for (int j = 0; j < kBinsPerThread; ++j) c[j] = 0u;
+      // this thread's kBinsPerThread consecutive bins as one 16-byte load per rank, all in flight
+      const int b0 = kBins - (tid + 1) * kBinsPerThread;
+      uint4 part[kMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r)
+        part[r] = r < static_cast<int>(cs) ? *reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, r) + b0)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) {
+        c[0] += part[r].w;       // bins in descending order: b0+3, b0+2, b0+1, b0
+        c[1] += part[r].z;
+        c[2] += part[r].y;
+        c[3] += part[r].x;
+      }
+      find_threshold_bin<kBinsPerThread>(c, kBins - 1 - tid * kBinsPerThread, k, warp_sums, &lvl_bin, &lvl_above,
+                                         &lvl_cnt);
+    }
+    __syncthreads();
+    bin_lo = lo + (lvl_bin << shift0);
+    const uint32_t bin_w1 = (1u << shift0) - 1u;
+    bin_hi = (hi - bin_lo) > bin_w1 ? bin_lo + bin_w1 : hi;
   }
-  __syncthreads();
   if (lvl_bin == kNotFound) {
     // The histogram holds fewer than top_k keys, which the row's data cannot produce:
     // record the fault and write nothing (every CTA of the cluster takes this branch).
@@ -337,9 +370,6 @@ topk_kernel(const TopkArgs a) {
     if (crank == 0 && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
     return;
   }
-  const uint32_t bin_lo = lo + (lvl_bin << shift0);
-  const uint32_t bin_w1 = (1u << shift0) - 1u;
-  const uint32_t bin_hi = (hi - bin_lo) > bin_w1 ? bin_lo + bin_w1 : hi;
   const uint32_t n_above_total = lvl_above, bcount = lvl_cnt;
   const uint32_t need0 = k - n_above_total;   // keys to take from the threshold bin
 
@@ -513,19 +543,6 @@ constexpr int kSubShift = kHistShift - 11;               // level-1 sub-bin widt
 constexpr int kSubCap = 1024;                            // sub-bin keys held in shared memory
 static_assert(kStreamEPT % 4 == 0 && kStreamPer0 % 4 == 0 && kStreamPer1 % 4 == 0, "chunk and histogram split");
 static_assert((1u << (kHistShift - kSubShift)) == static_cast<uint32_t>(kBins), "one level-1 bin per sub-bin");
-
-// PER consecutive bins starting at h, returned in descending bin order.
-template <int PER>
-__device__ __forceinline__ void load_bins_desc(const uint32_t* h, uint32_t (&c)[PER]) {
-#pragma unroll
-  for (int q = 0; q < PER / 4; ++q) {
-    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(h + 4 * q));
-    c[PER - 1 - 4 * q] = v.x;
-    c[PER - 2 - 4 * q] = v.y;
-    c[PER - 3 - 4 * q] = v.z;
-    c[PER - 4 - 4 * q] = v.w;
-  }
-}
 
 __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkArgs a) {
   __shared__ uint32_t hist[kBins];
