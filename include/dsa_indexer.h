@@ -137,7 +137,11 @@ DSA_API dsa_status_t dsa_quantize_rows_fp8(const void* src, dsa_dtype_t src_dtyp
  *   batch     host description; T_total = sum(q_lens)
  *   top_k     >= 1
  *   out_idx   device int32 [T_total, top_k]
- *   out_score device fp32  [T_total, top_k]
+ *   out_score device fp32  [T_total, top_k], or NULL when every sequence has seq_len <=
+ *             top_k: the short-sequence bypass ("Study MLA Indexer", 三个 why: with every
+ *             sequence within k the selection is the whole causal history and the scores
+ *             go unused), which launches no scoring kernel and writes out_idx[r] =
+ *             0 .. n_r - 1, then -1.  NULL with a longer sequence is DSA_ERR_INVALID_ARG.
  * Supported shapes: (H_I, d_I) = (64, 128) in bf16 or FP8, (4, 64) in bf16.
  */
 DSA_API dsa_status_t dsa_indexer_prefill(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,

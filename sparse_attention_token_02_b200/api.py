@@ -114,7 +114,8 @@ def dsa_quantize_rows_fp8(src: torch.Tensor, dst=None, scale=None, stream=None):
     return dst, scale
 
 
-def _run(fn_name, q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score, stream):
+def _run(fn_name, q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score, stream,
+         scores=True):
     b = _HostBatch(seq_lens, q_lens, k_base)
     T = b.total_q
     _require_cuda(w)
@@ -122,7 +123,7 @@ def _run(fn_name, q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx
         raise TypeError("w must be fp32")
     if out_idx is None:
         out_idx = torch.empty(T, top_k, dtype=torch.int32, device=q.device)
-    if out_score is None:
+    if out_score is None and scores:
         out_score = torch.empty(T, top_k, dtype=torch.float32, device=q.device)
     _require_cuda(out_idx, out_score)
     qq, kc = _query(q, q_scale), cache.c()
@@ -133,17 +134,20 @@ def _run(fn_name, q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx
 
 
 def dsa_indexer_prefill(q, cache: IndexerKCache, w, seq_lens, top_k, q_scale=None, q_lens=None, k_base=None,
-                        out_idx=None, out_score=None, stream=None):
-    """Scores + top-k for every query of a ragged batch; returns (out_idx int32, out_score fp32) [T_total, top_k]."""
+                        out_idx=None, out_score=None, stream=None, scores=True):
+    """Scores + top-k for every query of a ragged batch; returns (out_idx int32, out_score fp32) [T_total, top_k].
+    ``scores=False`` (every sequence at most top_k long): the short-sequence bypass, no scoring,
+    returns (out_idx, None)."""
     return _run("dsa_indexer_prefill", q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score,
-                stream)
+                stream, scores)
 
 
 def dsa_indexer_decode(q, cache: IndexerKCache, w, seq_lens, q_lens, top_k, q_scale=None, k_base=None,
-                       out_idx=None, out_score=None, stream=None):
-    """A decode step (1..4 queries per sequence at the end of each cache); returns (out_idx, out_score)."""
+                       out_idx=None, out_score=None, stream=None, scores=True):
+    """A decode step (1..4 queries per sequence at the end of each cache); returns (out_idx, out_score).
+    ``scores=False``: the short-sequence bypass, as for dsa_indexer_prefill."""
     return _run("dsa_indexer_decode", q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score,
-                stream)
+                stream, scores)
 
 
 def dsa_indexer_decode_noalloc(q, cache: IndexerKCache, w, seq_lens, q_lens, top_k, q_scale=None, k_base=None,

@@ -597,9 +597,13 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   if (mode == Mode::Scores) {
     if (!dense_out) return fail(DSA_ERR_INVALID_ARG, "out_scores is NULL");
     if (ld < v.max_seq_len || ld % 4) return fail(DSA_ERR_INVALID_ARG, "ld must be >= max(seq_lens) and a multiple of 4");
-  } else if (!out_idx || !out_score) {
-    return fail(DSA_ERR_INVALID_ARG, "out_idx / out_score is NULL");
+  } else if (!out_idx) {
+    return fail(DSA_ERR_INVALID_ARG, "out_idx is NULL");
+  } else if (!out_score && v.max_seq_len > top_k) {
+    return fail(DSA_ERR_INVALID_ARG, "out_score is NULL while a sequence is longer than top_k");
   }
+  // short-sequence bypass: no scores wanted and every row keeps its whole history
+  const bool bypass = mode != Mode::Scores && !out_score;
   const bool decode_sched = mode == Mode::Decode || (mode == Mode::Scores && v.max_q_len <= 4 &&
                                                      q->H_I == 64 && kc->d_I == 128);
   const int H = q->H_I, D = kc->d_I;
@@ -675,6 +679,18 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   char* mb = static_cast<char*>(c->cur_meta);
   const WsLayout wl = ws_layout(p.score_elems, v.total_q, p.stream_topk);
   char* wsb = reinterpret_cast<char*>(d_scores);
+  if (bypass) {
+    // every row holds at most top_k keys: the selection is its whole history, no scoring
+    TopkArgs s{};
+    s.row_pos = reinterpret_cast<const int32_t*>(mb + m.row_pos);
+    s.top_k = top_k;
+    s.out_idx = out_idx;
+    s.rows = reinterpret_cast<const int32_t*>(mb + m.topk_rows) + p.short_first;
+    s.n_rows = static_cast<int32_t>(p.short_count);
+    DSA_CUDA_TRY(launch_topk_short(s, stream), "top-k (short rows) launch");
+    ++g_launches;
+    return DSA_OK;
+  }
   uint32_t* d_hist = p.stream_topk ? reinterpret_cast<uint32_t*>(wsb + wl.hist) : nullptr;
   if (d_hist) DSA_CUDA_TRY(cudaMemsetAsync(d_hist, 0, wl.zero_bytes, stream), "cudaMemsetAsync");
 

@@ -1088,13 +1088,18 @@ __global__ void __launch_bounds__(kRowHistThreads) row_hist_kernel(const TopkArg
     if (h[b]) atomicAdd(row_hist + b, h[b]);
 }
 
-// Rows whose whole causal history fits in top_k: every position, then -1 / -inf.
+// Rows whose whole causal history fits in top_k: every position, then -1 / -inf.  Without
+// out_score (the short-sequence bypass) only the positions are written and no score is read.
 __global__ void __launch_bounds__(256) topk_short_kernel(const TopkArgs a) {
   grid_dependency_wait();                     // the scores come from the previous kernel
   const int row = a.rows[blockIdx.x];
   const int n = a.row_pos[row] + 1;
-  const float* src = a.scores + a.row_off[row];
   int32_t* oi = a.out_idx + static_cast<int64_t>(row) * a.top_k;
+  if (!a.out_score) {
+    for (int j = threadIdx.x; j < a.top_k; j += blockDim.x) oi[j] = j < n ? j : -1;
+    return;
+  }
+  const float* src = a.scores + a.row_off[row];
   float* os = a.out_score + static_cast<int64_t>(row) * a.top_k;
   for (int j = threadIdx.x; j < a.top_k; j += blockDim.x) {
     if (j < n) {

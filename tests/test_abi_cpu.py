@@ -69,6 +69,7 @@ def _batch(seq, ql=None, kb=None):
     ("decode_qlen", "INVALID_ARG"),
     ("dtype_mismatch", "INVALID_ARG"),
     ("misaligned", "INVALID_ARG"),
+    ("null_score_long_row", "INVALID_ARG"),
 ])
 def test_invalid_arguments_are_rejected_before_cuda(lib, case, expect):
     kc = _fake_cache()
@@ -97,8 +98,9 @@ def test_invalid_arguments_are_rejected_before_cuda(lib, case, expect):
         q.dtype = _lib.DSA_FP8_E4M3
     if case == "misaligned":
         q.data = 0x20004
+    out_score = None if case == "null_score_long_row" else ctypes.c_void_p(0x50000)   # bypass needs seq <= top_k
     st = fn(ctypes.byref(q), kc_p, ctypes.c_void_p(0x30000), ctypes.byref(b), top_k, ctypes.c_void_p(0x40000),
-            ctypes.c_void_p(0x50000), None)
+            out_score, None)
     assert _lib.STATUS_NAMES[st] == "DSA_ERR_" + expect, lib.dsa_get_last_error()
     assert lib.dsa_get_last_error()
 

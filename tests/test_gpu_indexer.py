@@ -230,6 +230,38 @@ def test_edge_top_k_larger_than_every_row_and_top_k_one():
     _check(up, idx1, sc1, list(range(wl.total_q)), top_k=1)
 
 
+@pytest.mark.parametrize("decode", [False, True])
+def test_short_sequence_bypass_writes_the_history_and_scores_nothing(decode):
+    # every sequence within top_k: no scoring kernel, out_idx = 0 .. n_r - 1 then -1
+    L, q_lens = (300, 7, 512), ((2, 1, 3) if decode else (300, 7, 512))
+    wl = W.scaled(W.decode() if decode else W.prefill(), seq_lens=L, q_lens=q_lens, top_k=512)
+    up = Uploaded(wl)
+    run = api.dsa_indexer_decode if decode else api.dsa_indexer_prefill
+    kw = dict(q_lens=q_lens) if not decode else {}
+    before = api.dsa_kernel_launch_count()
+    if decode:
+        idx, sc = run(up.q, up.cache, up.w, L, q_lens, wl.top_k, q_scale=up.q_scale, k_base=up.k_base, scores=False)
+    else:
+        idx, sc = run(up.q, up.cache, up.w, L, wl.top_k, q_scale=up.q_scale, k_base=up.k_base, scores=False, **kw)
+    api.dsa_check_device_errors()
+    assert sc is None and api.dsa_kernel_launch_count() - before == 1
+    idx = idx.cpu().numpy()
+    r = 0
+    for Lb, n in zip(L, q_lens):
+        for j in range(n):
+            hist = Lb - n + j + 1                             # the query's causal history
+            want = np.where(np.arange(wl.top_k) < hist, np.arange(wl.top_k), -1)
+            assert np.array_equal(idx[r], want), r
+            r += 1
+    # the same selection as the scored call, whose set is the whole history too
+    ref_i, _ = (run(up.q, up.cache, up.w, L, q_lens, wl.top_k, q_scale=up.q_scale, k_base=up.k_base) if decode else
+                run(up.q, up.cache, up.w, L, wl.top_k, q_scale=up.q_scale, k_base=up.k_base, **kw))
+    assert np.array_equal(np.sort(ref_i.cpu().numpy(), axis=1), np.sort(idx, axis=1))
+    with pytest.raises(RuntimeError, match="INVALID_ARG"):
+        run(up.q, up.cache, up.w, L, q_lens, 16, q_scale=up.q_scale, k_base=up.k_base, scores=False) if decode else \
+            run(up.q, up.cache, up.w, L, 16, q_scale=up.q_scale, k_base=up.k_base, scores=False, **kw)
+
+
 def test_edge_ties_and_zero_and_negative_weights():
     wl = W.scaled(W.prefill(), seq_lens=(1500,), q_lens=(1500,), top_k=100)
     inp = W.make_inputs(wl)
