@@ -403,9 +403,49 @@ def compressed_timings(api, hx, stream, dev, m=4, reps=10):
     kbytes = int(sum(blocks)) * wl.d * 2
     hbm = peaks()["hbm"]
     del cache, keys, flush
-    return {"m": m, "ms": ms, "pairs": pairs, "pairs_per_s": pairs / (ms * 1e-3),
-            "key_bytes": kbytes, "frac_of_hbm": kbytes / (ms * 1e-3) / 1e9 / hbm,
-            "note": "eager call (logits + top-k), one single-query decode row per query"}
+    out = {"m": m, "ms": ms, "pairs": pairs, "pairs_per_s": pairs / (ms * 1e-3),
+           "key_bytes": kbytes, "frac_of_hbm": kbytes / (ms * 1e-3) / 1e9 / hbm,
+           "note": "eager call (logits + top-k); the decode kernels with each query's limit at its last block"}
+    out["prefill"] = compressed_prefill_timing(api, stream, dev, m, reps)
+    return out
+
+
+def compressed_prefill_timing(api, stream, dev, m=4, reps=5, L=16384, H=64, d=128, top_k=2048):
+    """Prefill over an m-compressed cache: one sequence of L tokens, every token a query
+    (bf16, H_I = 64, d_I = 128, synthetic N(0, 1) block keys and queries, softmaxed w);
+    CUDA events around each call after a 256 MB L2-evicting read."""
+    import torch
+    nb = L // m
+    with torch.cuda.stream(stream):
+        cache = api.IndexerKCache.empty(nb, d, False, device=dev)
+        keys = torch.randn(nb, d, device=dev).to(torch.bfloat16)
+        api.dsa_indexer_kcache_append(cache, keys, torch.arange(nb, dtype=torch.int64, device=dev), stream=stream)
+        q = (torch.randn(L, H, d, device=dev) / d ** 0.5).to(torch.bfloat16)
+        w = torch.softmax(torch.randn(L, H, device=dev), dim=1)
+        flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        oi = torch.empty(L, top_k, dtype=torch.int32, device=dev)
+        os_ = torch.empty(L, top_k, dtype=torch.float32, device=dev)
+    call = lambda: api.dsa_indexer_prefill_compressed(q, cache, w, (L,), m, top_k, out_idx=oi, out_score=os_,
+                                                      stream=stream)
+    call()
+    total = 0.0
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            flush.max()
+            torch.cuda._sleep(_HOST_LEAD_CYCLES)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        stream.synchronize()
+        total += e0.elapsed_time(e1)
+    api.dsa_check_device_errors(stream)
+    ms = total / reps
+    pairs = sum((p + 1) // m for p in range(L))
+    flops = 2.0 * pairs * H * d
+    del cache, keys, q, flush
+    return {"L": L, "m": m, "ms": ms, "pairs": pairs, "pairs_per_s": pairs / (ms * 1e-3),
+            "tflops": flops / (ms * 1e-3) / 1e12, "note": "logits + top-k, causal over complete blocks"}
 
 
 class Harness:

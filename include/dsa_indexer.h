@@ -249,11 +249,22 @@ DSA_API dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const dsa_
  * A query at token position p sees the complete blocks j < floor((p + 1) / m): its own
  * still-open block is not scored (the sliding-window branch covers it).  out_idx holds
  * block indices j, out_score their scores; a query that sees no block gets only -1 / -inf.
- * Every q_lens[b] is at most 4 and every query is scored as its own single-query decode row.
+ * Every q_lens[b] is 1..4.  The decode kernels run unchanged with each query's causal limit
+ * moved to its last complete block; the queries of a sequence share every key tile.
  */
 DSA_API dsa_status_t dsa_indexer_decode_compressed(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
                                                    const dsa_batch_t* batch, int32_t m, int32_t top_k,
                                                    int32_t* out_idx, float* out_score, void* stream);
+
+/*
+ * Prefill over an m-compressed cache: the same arguments and visibility as
+ * dsa_indexer_decode_compressed, for any q_lens (0 .. seq_len, the queries at the last
+ * q_lens positions, as for dsa_indexer_prefill); the prefill kernels run with each query's
+ * causal limit moved to its last complete block.  out_score is required.
+ */
+DSA_API dsa_status_t dsa_indexer_prefill_compressed(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                                    const dsa_batch_t* batch, int32_t m, int32_t top_k,
+                                                    int32_t* out_idx, float* out_score, void* stream);
 
 /*
  * Rotary position embedding of indexer keys and queries, fused into the cache append and

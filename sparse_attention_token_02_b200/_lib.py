@@ -27,6 +27,7 @@ EXPORTED = (
     "dsa_indexer_decode_host",
     "dsa_indexer_decode_host_async",
     "dsa_indexer_decode_compressed",
+    "dsa_indexer_prefill_compressed",
     "dsa_indexer_kcache_append_rope",
     "dsa_rope_queries",
     "dsa_gather_rows",
@@ -100,6 +101,8 @@ def load() -> ctypes.CDLL:
     lib.dsa_indexer_decode_host_async.restype = st
     lib.dsa_indexer_decode_compressed.argtypes = [P(Query), P(KCache), V, P(Batch), I32, I32, V, V, V]
     lib.dsa_indexer_decode_compressed.restype = st
+    lib.dsa_indexer_prefill_compressed.argtypes = [P(Query), P(KCache), V, P(Batch), I32, I32, V, V, V]
+    lib.dsa_indexer_prefill_compressed.restype = st
     lib.dsa_indexer_kcache_append_rope.argtypes = [P(KCache), V, ctypes.c_int, V, V, I32, P(Rope), V]
     lib.dsa_indexer_kcache_append_rope.restype = st
     lib.dsa_rope_queries.argtypes = [V, ctypes.c_int, I64, I32, I32, V, P(Rope), V, ctypes.c_int, V, V]

@@ -219,6 +219,19 @@ def dsa_indexer_decode_compressed(q, cache: IndexerKCache, w, seq_lens, q_lens, 
                                   k_base=None, out_idx=None, out_score=None, stream=None):
     """Decode over an m-compressed key cache (block j of sequence b at cache row k_base[b] + j);
     seq_lens / q_lens in tokens.  Returns (block indices int32 [T, k], scores fp32 [T, k])."""
+    return _run_compressed("dsa_indexer_decode_compressed", q, cache, w, seq_lens, q_lens, m, top_k, q_scale, k_base,
+                           out_idx, out_score, stream)
+
+
+def dsa_indexer_prefill_compressed(q, cache: IndexerKCache, w, seq_lens, m, top_k, q_scale=None, q_lens=None,
+                                   k_base=None, out_idx=None, out_score=None, stream=None):
+    """Prefill over an m-compressed key cache (as dsa_indexer_decode_compressed, any q_lens;
+    None: every token of each sequence is a query)."""
+    return _run_compressed("dsa_indexer_prefill_compressed", q, cache, w, seq_lens, q_lens, m, top_k, q_scale, k_base,
+                           out_idx, out_score, stream)
+
+
+def _run_compressed(fn_name, q, cache, w, seq_lens, q_lens, m, top_k, q_scale, k_base, out_idx, out_score, stream):
     b = _HostBatch(seq_lens, q_lens, k_base)
     T = b.total_q
     _require_cuda(w)
@@ -228,8 +241,8 @@ def dsa_indexer_decode_compressed(q, cache: IndexerKCache, w, seq_lens, q_lens, 
         out_score = torch.empty(T, top_k, dtype=torch.float32, device=q.device)
     _require_cuda(out_idx, out_score)
     qq, kc = _query(q, q_scale), cache.c()
-    check(_lib.load().dsa_indexer_decode_compressed(ctypes.byref(qq), ctypes.byref(kc), _ptr(w), ctypes.byref(b.c),
-                                                    int(m), top_k, _ptr(out_idx), _ptr(out_score), _stream(stream)))
+    check(getattr(_lib.load(), fn_name)(ctypes.byref(qq), ctypes.byref(kc), _ptr(w), ctypes.byref(b.c), int(m), top_k,
+                                        _ptr(out_idx), _ptr(out_score), _stream(stream)))
     return out_idx, out_score
 
 

@@ -309,6 +309,9 @@ struct BatchView {
   int64_t total_q = 0;
   int32_t max_seq_len = 0;
   int32_t max_q_len = 0;
+  int32_t cmp = 1;              // 1: one cache row per token; m > 1: one per m tokens (compressed)
+  // keys a query at position p sees
+  int32_t visible(int32_t p) const { return (p + 1) / cmp; }
 };
 
 dsa_status_t check_cache(const dsa_kcache_t* kc) {
@@ -324,8 +327,10 @@ dsa_status_t check_cache(const dsa_kcache_t* kc) {
   return DSA_OK;
 }
 
-dsa_status_t check_batch(const dsa_batch_t* b, const dsa_kcache_t* kc, bool decode, BatchView* v) {
+dsa_status_t check_batch(const dsa_batch_t* b, const dsa_kcache_t* kc, bool decode, BatchView* v, int32_t cmp = 1) {
   if (!b) return fail(DSA_ERR_INVALID_ARG, "batch is NULL");
+  if (cmp < 1) return fail(DSA_ERR_INVALID_ARG, "m must be >= 1");
+  v->cmp = cmp;
   if (b->num_seqs < 0) return fail(DSA_ERR_INVALID_ARG, "num_seqs < 0");
   if (b->num_seqs > 0 && !b->seq_lens) return fail(DSA_ERR_INVALID_ARG, "batch.seq_lens is NULL");
   if (decode && b->num_seqs > 0 && !b->q_lens) return fail(DSA_ERR_INVALID_ARG, "decode needs batch.q_lens");
@@ -339,16 +344,17 @@ dsa_status_t check_batch(const dsa_batch_t* b, const dsa_kcache_t* kc, bool deco
     if (decode && (n < 1 || n > 4))
       return fail(DSA_ERR_INVALID_ARG, "decode: sequence %d has q_len %d, expected 1..4", i, n);
     const int64_t base = b->k_base ? b->k_base[i] : row;
-    if (base < 0 || base + L > kc->capacity_rows)
+    const int64_t rows = L / cmp;               // cache rows of the sequence
+    if (base < 0 || base + rows > kc->capacity_rows)
       return fail(DSA_ERR_INVALID_ARG, "sequence %d: rows [%lld, %lld) exceed the cache capacity %lld", i,
-                  static_cast<long long>(base), static_cast<long long>(base + L),
+                  static_cast<long long>(base), static_cast<long long>(base + rows),
                   static_cast<long long>(kc->capacity_rows));
     v->seq_len.push_back(L);
     v->q_len.push_back(n);
     v->k_base.push_back(base);
     v->q_off.push_back(qoff);
     qoff += n;
-    row += L;
+    row += rows;
     v->max_seq_len = std::max(v->max_seq_len, L);
     v->max_q_len = std::max(v->max_q_len, n);
   }
@@ -378,12 +384,13 @@ void plan_rows(const BatchView& v, bool dense, int64_t ld, Plan* p) {
     const int32_t pos0 = v.seq_len[b] - v.q_len[b];
     for (int j = 0; j < v.q_len[b]; ++j) {
       const int64_t r = v.q_off[b] + j;
-      p->row_pos[r] = pos0 + j;
+      const int32_t n = v.visible(pos0 + j);   // the row's keys (-1 below: none)
+      p->row_pos[r] = n - 1;
       if (dense) {
         p->row_off[r] = r * ld;
       } else {
         p->row_off[r] = off;
-        off += round_up(pos0 + j + 1, 4);
+        off += round_up(n, 4);
       }
     }
   }
@@ -404,7 +411,10 @@ void plan_prefill_items(const BatchView& v, int nt, int groups_per_item, int max
       it.n_tok = std::min(nt, v.q_len[b] - j);
       it.pos0 = pos0 + j;
       it.kt_begin = 0;
-      it.kt_end = static_cast<int32_t>((it.pos0 + it.n_tok + kKeyTile - 1) / kKeyTile);
+      const int32_t n_last = v.visible(it.pos0 + it.n_tok - 1);   // keys of the item's last query
+      if (n_last == 0) continue;                                   // no query of the item sees a key
+      it.kt_end = static_cast<int32_t>((n_last + kKeyTile - 1) / kKeyTile);
+      it.cmp = v.cmp;
       raw.push_back(it);
       const int groups = (it.n_tok + (nt / groups_per_item) - 1) / (nt / groups_per_item);
       cost.push_back(int64_t(it.kt_end) * (groups + 1));   // +1: the tile load and item overhead
@@ -438,7 +448,7 @@ void plan_decode_items(const BatchView& v, int max_ctas, Plan* p) {
   int64_t total = 0;
   std::vector<int32_t> tiles(v.num_seqs);
   for (int b = 0; b < v.num_seqs; ++b) {
-    tiles[b] = (v.seq_len[b] + kKeyTile - 1) / kKeyTile;
+    tiles[b] = (v.visible(v.seq_len[b] - 1) + kKeyTile - 1) / kKeyTile;   // the last query sees the most
     if (v.q_len[b] == 0) tiles[b] = 0;
     total += tiles[b];
   }
@@ -464,6 +474,7 @@ void plan_decode_items(const BatchView& v, int max_ctas, Plan* p) {
       it.pos0 = v.seq_len[b] - v.q_len[b];
       it.kt_begin = t;
       it.kt_end = t + take;
+      it.cmp = v.cmp;
       p->items.push_back(it);
       t += take;
       quota -= take;
@@ -583,12 +594,14 @@ enum class Mode { Prefill, Decode, Scores };
 
 dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
                          const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx, float* out_score,
-                         float* dense_out, int64_t ld, void* stream_v) {
+                         float* dense_out, int64_t ld, void* stream_v, int32_t cmp = 1) {
   g_last_error.clear();
   dsa_status_t st = check_cache(kc);
   if (st != DSA_OK) return st;
   BatchView v;
-  if ((st = check_batch(batch, kc, mode == Mode::Decode, &v)) != DSA_OK) return st;
+  if ((st = check_batch(batch, kc, mode == Mode::Decode, &v, cmp)) != DSA_OK) return st;
+  if (cmp > 1 && (mode == Mode::Scores || !out_score))
+    return fail(DSA_ERR_INVALID_ARG, "a compressed cache needs the scores and the selection");
   if (mode != Mode::Scores && top_k < 1) return fail(DSA_ERR_INVALID_ARG, "top_k must be >= 1");
   if (v.total_q == 0) return DSA_OK;          // nothing to score: no pointer is touched
   if ((st = check_query(q, kc)) != DSA_OK) return st;
@@ -630,7 +643,7 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   // The plan depends only on the batch description, so a repeated batch reuses the
   // tables already on the device (decode loops, graph capture).
   std::vector<int64_t> key = {static_cast<int64_t>(mode), H, D, fp8, top_k, ld, v.num_seqs,
-                              reinterpret_cast<int64_t>(c->user_ws)};
+                              reinterpret_cast<int64_t>(c->user_ws), v.cmp};
   for (int b = 0; b < v.num_seqs; ++b) {
     key.push_back(v.seq_len[b]);
     key.push_back(v.q_len[b]);
@@ -1000,56 +1013,27 @@ dsa_status_t dsa_indexer_decode_host_async(const dsa_query_t* q, const dsa_kcach
                           out_score_host, stream_v, static_cast<cudaEvent_t>(done_event), false);
 }
 
+// Over a cache of one key per m tokens the same kernels run with every query's causal limit
+// mapped to the blocks its position completes (the logits epilogue masks keys past
+// (p + 1) / m - 1, the planner sizes key ranges and score rows by it).
 dsa_status_t dsa_indexer_decode_compressed(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
                                            const dsa_batch_t* batch, int32_t m, int32_t top_k, int32_t* out_idx,
                                            float* out_score, void* stream_v) {
-  g_last_error.clear();
-  if (!q || !kc || !w || !batch || !out_idx || !out_score) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (m < 1 || top_k < 1) return fail(DSA_ERR_INVALID_ARG, "m and top_k must be >= 1");
-  if (batch->num_seqs < 0 || (batch->num_seqs > 0 && (!batch->seq_lens || !batch->q_lens)))
-    return fail(DSA_ERR_INVALID_ARG, "decode needs batch.seq_lens and batch.q_lens");
-  if (q->dtype != DSA_BF16 && q->dtype != DSA_FP8_E4M3) return fail(DSA_ERR_INVALID_ARG, "q->dtype must be DSA_BF16 or DSA_FP8_E4M3");
-  // every query becomes a single-query decode row over its visible blocks
-  std::vector<int32_t> vis;
-  std::vector<int64_t> base;
-  int64_t packed = 0;
-  for (int b = 0; b < batch->num_seqs; ++b) {
-    const int32_t L = batch->seq_lens[b], n = batch->q_lens[b];
-    if (L < 0 || n < 0 || n > L || n > 4) return fail(DSA_ERR_INVALID_ARG, "sequence %d: need 0 <= q_len <= min(4, seq_len)", b);
-    const int64_t kb = batch->k_base ? batch->k_base[b] : packed;
-    packed += L / m;
-    for (int32_t j = 0; j < n; ++j) {
-      vis.push_back((L - n + j + 1) / m);
-      base.push_back(kb);
-    }
+  if (m < 1) {
+    g_last_error.clear();
+    return fail(DSA_ERR_INVALID_ARG, "m must be >= 1");
   }
-  const int64_t T = static_cast<int64_t>(vis.size());
-  const size_t q_row = size_t(q->H_I) * q->d_I * (q->dtype == DSA_FP8_E4M3 ? 1 : 2);
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-  dsa_status_t st;
-  // runs of rows that see at least one block go through the decode path; the rest are padding
-  for (int64_t r0 = 0; r0 < T;) {
-    int64_t r1 = r0;
-    const bool any = vis[r0] > 0;
-    while (r1 < T && (vis[r1] > 0) == any) ++r1;
-    if (any) {
-      const std::vector<int32_t> ones(size_t(r1 - r0), 1);
-      dsa_batch_t pb{static_cast<int32_t>(r1 - r0), vis.data() + r0, ones.data(), base.data() + r0};
-      dsa_query_t qr = *q;
-      qr.data = static_cast<const char*>(q->data) + r0 * q_row;
-      qr.scale = q->scale ? q->scale + r0 : nullptr;
-      if ((st = dsa_indexer_decode(&qr, kc, w + r0 * q->H_I, &pb, top_k, out_idx + r0 * top_k,
-                                   out_score + r0 * top_k, stream_v)) != DSA_OK)
-        return st;
-    } else {
-      const int64_t cnt = (r1 - r0) * top_k;
-      DSA_CUDA_TRY(cudaMemsetAsync(out_idx + r0 * top_k, 0xFF, size_t(cnt) * sizeof(int32_t), stream), "cudaMemsetAsync");
-      DSA_CUDA_TRY(launch_fill_f32(out_score + r0 * top_k, cnt, -INFINITY, stream), "fill kernel launch");
-      ++g_launches;
-    }
-    r0 = r1;
+  return run_indexer(Mode::Decode, q, kc, w, batch, top_k, out_idx, out_score, nullptr, 0, stream_v, m);
+}
+
+dsa_status_t dsa_indexer_prefill_compressed(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
+                                            const dsa_batch_t* batch, int32_t m, int32_t top_k, int32_t* out_idx,
+                                            float* out_score, void* stream_v) {
+  if (m < 1) {
+    g_last_error.clear();
+    return fail(DSA_ERR_INVALID_ARG, "m must be >= 1");
   }
-  return DSA_OK;
+  return run_indexer(Mode::Prefill, q, kc, w, batch, top_k, out_idx, out_score, nullptr, 0, stream_v, m);
 }
 
 dsa_status_t dsa_selftest_wait_expiry(int64_t limit_cycles, void* stream_v) {

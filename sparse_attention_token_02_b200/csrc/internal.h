@@ -49,7 +49,8 @@ struct LogitsItem {
   int32_t pos0;      // position of the first query inside its sequence
   int32_t kt_begin;  // first key tile
   int32_t kt_end;    // one past the last key tile
-  int32_t pad;
+  int32_t cmp;       // 0 or 1: the cache holds every key; m > 1: one key per m tokens (query at
+                     // position p sees keys 0 .. (p + 1) / m - 1)
 };
 static_assert(sizeof(LogitsItem) == 32, "LogitsItem layout");
 

@@ -419,7 +419,11 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
         }
       }
       const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
-      const int pos_last = wi.pos0 + wi.n_tok - 1;
+      // last key query j sees: its position, or over a cache of one key per `cmp` tokens the
+      // last block its position completes
+      const int cmp = wi.cmp > 1 ? wi.cmp : 1;
+      auto last_key = [&](int j) -> int { return cmp == 1 ? wi.pos0 + j : (wi.pos0 + j + 1) / cmp - 1; };
+      const int pos_last = last_key(wi.n_tok - 1);
       // FP8 key scales are loaded kScalePrefetch tiles ahead of use, so the per-tile
       // global-memory latency overlaps the epilogues of the tiles in between.
       constexpr int PF = kScalePrefetch;
@@ -456,7 +460,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
           const int j_hi = min(j_lo + C::TPA, wi.n_tok);
           if constexpr (C::ONE_QUERY_PER_WARP) {
             const int j = part;                                        // this warp's query
-            if (j < wi.n_tok && key0 <= wi.pos0 + j) {                 // warp-uniform
+            if (j < wi.n_tok && key0 <= last_key(j)) {                 // warp-uniform
               float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #if DSA_TMEM_X64
               uint32_t r[64];
@@ -473,7 +477,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
               relu_wsum32_reg(r1, wr_hi, a0, a1);
 #endif
               const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
-              const bool valid = key <= wi.pos0 + j;
+              const bool valid = key <= last_key(j);
               if (valid) args.scores[rowoff[j] + key] = v;
               if (C::HIST && args.row_hist) hist_count(j, v, valid);
             }
@@ -481,7 +485,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
             // many epilogue warps: one 32-column chunk in registers at a time
             constexpr int CPT = C::H / 32;
             for (int j = j_lo + part; j < j_hi; j += SPLIT) {
-              if (key0 > wi.pos0 + j) continue;                        // the tile is after this query
+              if (key0 > last_key(j)) continue;                        // the tile is after this query
               float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
               for (int c = 0; c < CPT; ++c) {
@@ -491,7 +495,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
                 relu_wsum32(r, wq + j * C::H + c * 32, a0, a1);
               }
               const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
-              const bool valid = key <= wi.pos0 + j;
+              const bool valid = key <= last_key(j);
               if (valid) args.scores[rowoff[j] + key] = v;
               if (C::HIST && args.row_hist) hist_count(j, v, valid);
             }
@@ -505,7 +509,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
 #pragma unroll
               for (int u = 0; u < C::QB; ++u) {
                 const int j = j0 + u * SPLIT;
-                live[u] = j < j_hi && key0 <= wi.pos0 + j;             // warp-uniform
+                live[u] = j < j_hi && key0 <= last_key(j);             // warp-uniform
                 any |= live[u];
                 if (live[u]) {
 #pragma unroll
@@ -519,7 +523,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
                 const int j = j0 + u * SPLIT;
                 if (live[u]) {
                   const float v = relu_wsum<CPT>(r[u], wq + j * C::H) * kscale;
-                  const bool valid = key <= wi.pos0 + j;
+                  const bool valid = key <= last_key(j);
                   if (valid) args.scores[rowoff[j] + key] = v;
                   if (C::HIST && args.row_hist) hist_count(j, v, valid);
                 }
@@ -543,7 +547,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
                   for (int h = 0; h < C::H; ++h)
                     acc = fmaf(wq[j * C::H + h], fmaxf(__uint_as_float(r[u * C::H + h]), 0.f), acc);
                   const float v = acc * kscale;
-                  const bool valid = key <= wi.pos0 + j;
+                  const bool valid = key <= last_key(j);
                   if (valid) args.scores[rowoff[j] + key] = v;
                   if (C::HIST && args.row_hist) hist_count(j, v, valid);
                 }
