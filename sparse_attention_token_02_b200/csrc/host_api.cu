@@ -678,6 +678,12 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     const size_t ws_bytes = ws_layout(np.score_elems, v.total_q, np.stream_topk).total;
     if ((st = reserve(c, nm.total, ws_bytes, &dm, &ds)) != DSA_OK) return st;
     if ((st = stage_upload(c, blob.data(), blob.size(), dm)) != DSA_OK) return st;
+    if (np.stream_topk) {
+      // the histograms and row counters start clear; from then on the top-k kernels clear
+      // each row's after use, so a repeated call needs no memset between its launches
+      const WsLayout nw = ws_layout(np.score_elems, v.total_q, true);
+      DSA_CUDA_TRY(cudaMemsetAsync(reinterpret_cast<char*>(ds) + nw.hist, 0, nw.zero_bytes, stream), "cudaMemsetAsync");
+    }
     c->plan = std::move(np);
     c->layout = nm;
     c->plan_key = key;
@@ -705,7 +711,12 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     return DSA_OK;
   }
   uint32_t* d_hist = p.stream_topk ? reinterpret_cast<uint32_t*>(wsb + wl.hist) : nullptr;
-  if (d_hist) DSA_CUDA_TRY(cudaMemsetAsync(d_hist, 0, wl.zero_bytes, stream), "cudaMemsetAsync");
+  // from the scoring launch on, a failed enqueue leaves histograms uncleared: plan afresh next time
+  struct Replan {
+    Ctx* c;
+    bool armed;
+    ~Replan() { if (armed) c->meta_valid = false; }
+  } replan{c, d_hist != nullptr};
 
   CUtensorMap tk, tq;
   if ((st = encode_rows(&tk, kc->k, fp8, kc->capacity_rows, D, kKeyTile)) != DSA_OK) return st;
@@ -748,6 +759,7 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     TopkArgs s = ta;
     s.rows = rows + p.short_first;
     s.n_rows = static_cast<int32_t>(p.short_count);
+    s.row_hist = d_hist;                      // decode: cleared for the next call
     DSA_CUDA_TRY(launch_topk_short(s, stream), "top-k (short rows) launch");
     ++g_launches;
   }
@@ -784,6 +796,7 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     ++g_launches;
   }
   if (g_prof[2]) DSA_CUDA_TRY(cudaEventRecordWithFlags(g_prof[2], stream, ev_flags), "cudaEventRecord");
+  replan.armed = false;
   return DSA_OK;
 }
 

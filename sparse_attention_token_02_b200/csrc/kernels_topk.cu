@@ -124,6 +124,17 @@ __device__ __forceinline__ void load_bins_desc(const uint32_t* h, uint32_t (&c)[
   }
 }
 
+// Zeroes part `part` of `parts` of a row's coarse histogram (16-byte stores) once every
+// reader of it is done, so the next call's logits epilogue counts into a clear histogram
+// without a memset between the launches.
+__device__ __forceinline__ void clear_row_hist(uint32_t* h, int part, int parts) {
+  constexpr int kVecs = kHistBins / 4;
+  uint4* v = reinterpret_cast<uint4*>(h);
+  const int per = (kVecs + parts - 1) / parts;
+  for (int i = part * per + static_cast<int>(threadIdx.x); i < min(kVecs, (part + 1) * per); i += blockDim.x)
+    v[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // Calls f(key, index, valid) for candidates [0, m), each thread taking every NT-th one
 // (valid is false past m).  Reads
 // go in batches of CPT per thread, all loads of a batch issued before any is used: global
@@ -363,10 +374,14 @@ topk_kernel(const TopkArgs a) {
     const uint32_t bin_w1 = (1u << shift0) - 1u;
     bin_hi = (hi - bin_lo) > bin_w1 ? bin_lo + bin_w1 : hi;
   }
+  // the row's coarse histogram, cleared by the cluster after its first cluster-wide barrier
+  // (every CTA has read it by then)
+  uint32_t* my_hist = a.row_hist ? const_cast<uint32_t*>(a.row_hist) + static_cast<int64_t>(row) * kHistBins : nullptr;
   if (lvl_bin == kNotFound) {
     // The histogram holds fewer than top_k keys, which the row's data cannot produce:
     // record the fault and write nothing (every CTA of the cluster takes this branch).
     cluster.sync();                           // no CTA still reads another's shared memory
+    if (my_hist) clear_row_hist(my_hist, crank, cs);
     if (crank == 0 && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
     return;
   }
@@ -412,6 +427,7 @@ topk_kernel(const TopkArgs a) {
       }
     }
     cluster.sync();                           // rank 0 holds the whole bin; counters are final
+    if (my_hist) clear_row_hist(my_hist, crank, cs);
     if (crank != 0) return;                   // nobody reads another CTA's memory after this point
     const bool above_ok = cnt_above == n_above_total && cnt_cand == bcount;
     const bool ok = rank0_select<false, kThreads>(cand_key, cand_idx, bcount, 0u, bin_lo, bin_hi, need0, n_above_total, oi, os, hist,
@@ -429,6 +445,8 @@ topk_kernel(const TopkArgs a) {
   s.hi = bin_hi;
   s.need = need0;
   s.done = 0;
+  cluster.sync();                             // every CTA has read the coarse histogram
+  if (my_hist) clear_row_hist(my_hist, crank, cs);
   for (int level = 0; level < 8; ++level) {
     if (s.lo == s.hi) { s.done = 2; break; }
     const int bits = 32 - __clz(s.hi - s.lo);
@@ -564,6 +582,13 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
   // row counters: [0] bin keys gathered, [1] keys written above the bin (one 64-bit word), [2] chunks done
   uint32_t* ctr = a.row_ctr + 4 * static_cast<int64_t>(row);
   uint32_t* sub_hist = a.row_hist1 + static_cast<int64_t>(row) * kBins;
+  // the CTA that takes the row's last ticket leaves the row's histograms and counters clear
+  // for the next call (every other CTA of the row has read them before its ticket)
+  auto clear_row_state = [&]() {
+    clear_row_hist(const_cast<uint32_t*>(a.row_hist) + static_cast<int64_t>(row) * kHistBins, 0, 1);
+    for (int b = tid; b < kBins; b += kStreamThreads) sub_hist[b] = 0u;
+    if (tid < 4) ctr[tid] = 0u;
+  };
   if (tid == 0) lvl_bin = kNotFound;          // published by the scan's barriers below
   grid_dependency_wait();                     // scores and histograms come from the previous kernel
 
@@ -585,8 +610,16 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
   __syncthreads();
   if (lvl_bin == kNotFound) {
     // fewer than top_k keys counted for a row longer than top_k: every CTA of the row
-    // lands here, so no CTA of it takes the ticket and nothing is written
-    if (tid == 0 && ch.begin == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    // lands here; nothing is written, the last one clears the row's state
+    if (tid == 0) {
+      if (ch.begin == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+      is_last = atomicAdd(ctr + 2, 1u) == static_cast<uint32_t>(ch.n_chunks - 1);
+    }
+    __syncthreads();
+    if (is_last) {
+      __threadfence();
+      clear_row_state();
+    }
     return;
   }
   const uint32_t bin_lo = lvl_bin << kHistShift;
@@ -651,6 +684,8 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
   const unsigned long long got = __ldcg(reinterpret_cast<const unsigned long long*>(ctr));
   if (static_cast<uint32_t>(got >> 32) != n_above_total || static_cast<uint32_t>(got) != bcount) {
     if (tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    __syncthreads();                          // every thread has read the counters
+    clear_row_state();
     return;
   }
   const uint32_t need0 = k - n_above_total;
@@ -662,6 +697,7 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
   __syncthreads();
   if (lvl_bin == kNotFound) {
     if (tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+    clear_row_state();
     return;
   }
   const uint32_t above1 = lvl_above, cnt1 = lvl_cnt;
@@ -704,6 +740,7 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
                                             &ctr_a, &ctr_b);
   }
   if (!ok && tid == 0) record_error(a.err, DSA_DEVERR_TOPK, row);
+  clear_row_state();                          // the level-1 counts were read before the select
 }
 
 // ---- row-streaming top-k (prefill: many rows, no histogram from the logits kernel).
@@ -1095,6 +1132,8 @@ __global__ void __launch_bounds__(256) topk_short_kernel(const TopkArgs a) {
   const int row = a.rows[blockIdx.x];
   const int n = a.row_pos[row] + 1;
   int32_t* oi = a.out_idx + static_cast<int64_t>(row) * a.top_k;
+  // decode: the logits epilogue counted this row too; leave its histogram clear for the next call
+  if (a.row_hist) clear_row_hist(const_cast<uint32_t*>(a.row_hist) + static_cast<int64_t>(row) * kHistBins, 0, 1);
   if (!a.out_score) {
     for (int j = threadIdx.x; j < a.top_k; j += blockDim.x) oi[j] = j < n ? j : -1;
     return;
