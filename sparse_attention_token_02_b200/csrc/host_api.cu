@@ -483,12 +483,12 @@ void plan_decode_items(const BatchView& v, int max_ctas, Plan* p) {
   }
 }
 
-dsa_status_t plan_topk(const BatchView& v, int top_k, int sms, Plan* p) {
+dsa_status_t plan_topk(const BatchView& v, int top_k, int sms, Plan* p, int max_cs = 8) {
   std::vector<int32_t> shorts, longs;
   for (int64_t r = 0; r < v.total_q; ++r) (p->row_pos[r] + 1 <= top_k ? shorts : longs).push_back(static_cast<int32_t>(r));
   const int64_t n_long = static_cast<int64_t>(longs.size());
   int cs_par = 1;
-  if (n_long > 0 && n_long < 2 * sms) cs_par = std::min(8, next_pow2((2 * sms + n_long - 1) / n_long));
+  if (n_long > 0 && n_long < 2 * sms) cs_par = std::min(max_cs, next_pow2((2 * sms + n_long - 1) / n_long));
   std::map<std::pair<int, int>, std::vector<int32_t>> cls;
   for (int32_t r : longs) {
     const int64_t n = int64_t(p->row_pos[r]) + 1;
@@ -516,18 +516,23 @@ dsa_status_t plan_topk(const BatchView& v, int top_k, int sms, Plan* p) {
 }
 
 // Decode rows: chunks of kStreamChunk keys for the streaming top-k (no length limit).
-// Decode rows (the coarse histograms given).  A bf16 batch whose rows are at most 65536
+// Decode rows (the coarse histograms given).  A bf16 batch whose rows are at most 32768
 // keys long takes one cluster per row (the cluster kernel seeded by the histogram: no
-// global counters, fence or ticket between the CTAs of a row; 14.3 us against 16.2 us for
-// the decode batch); FP8 batches and longer rows stream 4096-key chunks (the FP8 histogram
-// pass needs those chunks anyway, and 32 keys a thread leave the clusters slower there).
+// global counters, fence or ticket between the CTAs of a row); FP8 batches and longer rows
+// stream 4096-key chunks (the FP8 histogram pass needs those chunks anyway, and 32 keys a
+// thread leave the clusters slower there).
 void plan_topk_stream(const BatchView& v, int top_k, int sms, bool fp8, Plan* p) {
   p->topk_rows.clear();
   p->classes.clear();
   p->chunks.clear();
   int64_t longest = 0;
   for (int64_t r = 0; r < v.total_q; ++r) longest = std::max(longest, int64_t(p->row_pos[r]) + 1);
-  p->cluster_topk = !fp8 && longest <= int64_t(8) * 16 * kTopkThreads && plan_topk(v, top_k, sms, p) == DSA_OK;
+  // clusters of at most 4 CTAs: they find room on the SMs the logits kernel frees as it drains
+  // (the step overlaps better: 55.5-56.6 us against 60.0 us with clusters of 8), and rows up
+  // to 4 x 16 x 512 keys keep 16 keys a thread
+  constexpr int kMaxCs = 4;
+  p->cluster_topk = !fp8 && longest <= int64_t(kMaxCs) * 16 * kTopkThreads &&
+                    plan_topk(v, top_k, sms, p, kMaxCs) == DSA_OK;
   if (p->cluster_topk) return;
   p->topk_rows.clear();
   p->classes.clear();
