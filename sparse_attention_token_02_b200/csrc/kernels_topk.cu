@@ -33,7 +33,6 @@ namespace dsa {
 namespace {
 
 constexpr int kThreads = kTopkThreads;
-constexpr int kWarps = kThreads / 32;
 constexpr int kBins = kTopkBins;
 constexpr int kBinsPerThread = kBins / kThreads;
 static_assert(kBins % kThreads == 0, "bins per thread");
