@@ -14,8 +14,10 @@
  * ---------------------------------------
  * - Pointers named "device" are CUDA device pointers on the current device;
  *   "host" pointers are read synchronously during the call and may be reused
- *   as soon as it returns.  Device pointers passed to the tensor-core path (the
- *   cache, the queries) must be 16-byte aligned.
+ *   as soon as it returns -- except the *_host buffers of the host-step calls
+ *   (dsa_indexer_decode_host and _async), which are copied asynchronously and
+ *   stay in use until the step completes.  Device pointers passed to the
+ *   tensor-core path (the cache, the queries) must be 16-byte aligned.
  * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
  *   only enqueues work on it; outputs are valid once the stream has reached
  *   that point.  Calls that share a stream may be issued back to back.
