@@ -141,7 +141,7 @@ def compressed_visible(position: int, m: int) -> int:
 
 
 def decode_compressed_oracle(q, kc_seqs, w, seq_lens, q_lens, m: int, top_k: int) -> dict:
-    """Decode over an m-compressed key cache.
+    """Decode (or prefill: q_lens up to seq_lens) over an m-compressed key cache.
 
     kc_seqs[b]: [floor(seq_lens[b] / m), d] fp64 compressed keys of sequence b (block j covers
     tokens j*m .. j*m + m - 1); seq_lens / q_lens in tokens, queries at the last q_lens
