@@ -262,6 +262,39 @@ def test_short_sequence_bypass_writes_the_history_and_scores_nothing(decode):
             run(up.q, up.cache, up.w, L, 16, q_scale=up.q_scale, k_base=up.k_base, scores=False, **kw)
 
 
+@pytest.mark.parametrize("decode", [False, True])
+def test_caller_workspace_gives_the_same_selection_and_refuses_a_short_one(decode):
+    L, q_lens = (3000, 2049, 700), ((2, 1, 1) if decode else (3000, 2049, 700))
+    wl = W.scaled(W.decode() if decode else W.prefill(), seq_lens=L, q_lens=q_lens, top_k=512, seed=95)
+    up = Uploaded(wl)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ref_i, ref_s = _run(up, decode=decode)
+        need = api.dsa_indexer_workspace_bytes(up.q, L, wl.top_k, q_lens=q_lens)
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        try:
+            api.dsa_set_workspace(ws, stream=s)
+            if decode:
+                idx, sc = api.dsa_indexer_decode(up.q, up.cache, up.w, L, q_lens, wl.top_k, q_scale=up.q_scale,
+                                                 k_base=up.k_base, stream=s)
+            else:
+                idx, sc = api.dsa_indexer_prefill(up.q, up.cache, up.w, L, wl.top_k, q_scale=up.q_scale, q_lens=q_lens,
+                                                  k_base=up.k_base, stream=s)
+            api.dsa_check_device_errors(s)
+            for (gi, gs), (ri, rs) in zip(_sorted_rows(idx.cpu().numpy(), sc.cpu().numpy()), _sorted_rows(ref_i, ref_s)):
+                assert np.array_equal(gi, ri)
+                np.testing.assert_array_equal(gs, rs)
+            api.dsa_set_workspace(ws[: 1 << 12], stream=s)       # far too small
+            with pytest.raises(RuntimeError, match="ALLOC"):
+                api.dsa_indexer_decode(up.q, up.cache, up.w, L, q_lens, wl.top_k, q_scale=up.q_scale,
+                                       k_base=up.k_base, stream=s) if decode else \
+                    api.dsa_indexer_prefill(up.q, up.cache, up.w, L, wl.top_k, q_scale=up.q_scale, q_lens=q_lens,
+                                            k_base=up.k_base, stream=s)
+        finally:
+            api.dsa_set_workspace(None, stream=s)
+        s.synchronize()
+
+
 def test_edge_ties_and_zero_and_negative_weights():
     wl = W.scaled(W.prefill(), seq_lens=(1500,), q_lens=(1500,), top_k=100)
     inp = W.make_inputs(wl)
