@@ -75,7 +75,9 @@ def _query(q: torch.Tensor, q_scale) -> Query:
 
 
 class _HostBatch:
-    """Keeps the host arrays of a dsa_batch_t alive for the duration of a call."""
+    """Keeps the host arrays of a dsa_batch_t alive for the duration of a call.  Built once
+    with host_batch() it can be passed in place of ``seq_lens`` to the calls that take one,
+    so a loop over steps with the same batch does not convert the lists every step."""
 
     def __init__(self, seq_lens, q_lens, k_base):
         self.seq = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
@@ -88,6 +90,19 @@ class _HostBatch:
     @property
     def total_q(self) -> int:
         return int(self.seq.sum() if self.ql is None else self.ql.sum())
+
+
+def host_batch(seq_lens, q_lens=None, k_base=None) -> _HostBatch:
+    """A reusable batch description (seq_lens, q_lens, k_base as for the calls)."""
+    return _HostBatch(seq_lens, q_lens, k_base)
+
+
+def _batch(seq_lens, q_lens, k_base) -> _HostBatch:
+    if isinstance(seq_lens, _HostBatch):
+        if q_lens is not None or k_base is not None:
+            raise ValueError("pass q_lens / k_base to host_batch(), not with a prebuilt batch")
+        return seq_lens
+    return _HostBatch(seq_lens, q_lens, k_base)
 
 
 def dsa_indexer_kcache_append(cache: IndexerKCache, k_new: torch.Tensor, dst_rows: torch.Tensor, stream=None):
@@ -116,7 +131,7 @@ def dsa_quantize_rows_fp8(src: torch.Tensor, dst=None, scale=None, stream=None):
 
 def _run(fn_name, q, q_scale, cache, w, seq_lens, q_lens, k_base, top_k, out_idx, out_score, stream,
          scores=True):
-    b = _HostBatch(seq_lens, q_lens, k_base)
+    b = _batch(seq_lens, q_lens, k_base)
     T = b.total_q
     _require_cuda(w)
     if w.dtype != torch.float32:
@@ -180,7 +195,8 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
     upload the new keys (bf16 or fp32 [n_new, d_I], cache rows ``dst_rows_host`` int64), queries
     [T, H_I, d_I] (bf16, or uint8 E4M3 codes with ``q_scale_host``) and weights [T, H_I] fp32,
     append, score + select, and copy the selection into ``out_idx_host`` int32 / ``out_score_host``
-    fp32 [T, top_k].  Returns at once; the host outputs are complete when ``stream`` has finished,
+    fp32 [T, top_k].  ``seq_lens`` may be a prebuilt host_batch() (q_lens and k_base then None).
+    Returns at once; the host outputs are complete when ``stream`` has finished,
     or, with ``done_event`` (a torch.cuda.Event; dsa_indexer_decode_host_async), once that event
     has completed, while ``stream`` goes on without waiting for the read-back.  Pinned host
     tensors keep the copies asynchronous."""
@@ -193,7 +209,7 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
         raise TypeError("dst_rows must be int64")
     if q_host.dim() != 3:
         raise ValueError("q must be [T_total, H_I, d_I]")
-    b = _HostBatch(seq_lens, q_lens, k_base)
+    b = _batch(seq_lens, q_lens, k_base)
     qq = Query(q_host.data_ptr(), q_scale_host.data_ptr() if q_scale_host is not None else None, _dtype_code(q_host),
                q_host.shape[1], q_host.shape[2])
     kc = cache.c()

@@ -128,3 +128,14 @@ def test_wait_expiry_self_test_checks_its_limit(lib):
     for bad in (0, -5, 3_000_000_000):
         st = lib.dsa_selftest_wait_expiry(bad, None)
         assert _lib.STATUS_NAMES[st] == "DSA_ERR_INVALID_ARG", lib.dsa_get_last_error()
+
+
+def test_prebuilt_host_batch_is_used_as_given():
+    from sparse_attention_token_02_b200 import api
+    hb = api.host_batch([300, 7], [2, 1], [0, 400])
+    assert api._batch(hb, None, None) is hb
+    assert hb.total_q == 3 and hb.c.num_seqs == 2
+    with pytest.raises(ValueError, match="host_batch"):
+        api._batch(hb, [2, 1], None)
+    fresh = api._batch([300, 7], None, None)
+    assert fresh.total_q == 307 and fresh.ql is None
