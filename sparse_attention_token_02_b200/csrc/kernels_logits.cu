@@ -25,6 +25,8 @@
 // the MMAs of the next.  Every wait is bounded (see ptx.cuh).
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -422,8 +424,7 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
       // last key query j sees: its position, or over a cache of one key per `cmp` tokens the
       // last block its position completes
       const int cmp = wi.cmp > 1 ? wi.cmp : 1;
-      auto last_key = [&](int j) -> int { return cmp == 1 ? wi.pos0 + j : (wi.pos0 + j + 1) / cmp - 1; };
-      const int pos_last = last_key(wi.n_tok - 1);
+      const int pos_last = cmp == 1 ? wi.pos0 + wi.n_tok - 1 : (wi.pos0 + wi.n_tok) / cmp - 1;
       // FP8 key scales are loaded kScalePrefetch tiles ahead of use, so the per-tile
       // global-memory latency overlaps the epilogues of the tiles in between.
       constexpr int PF = kScalePrefetch;
@@ -437,131 +438,144 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
 #pragma unroll
         for (int i = 0; i < PF; ++i) ks_ring[i] = load_scale(wi.kt_begin + i);
       }
-      for (int kt = wi.kt_begin; kt < wi.kt_end && ok; ++kt) {
-        const int key0 = kt * C::BM;                      // first key of the tile
-        const int key = key0 + sub * 32 + lane;           // this thread's key (its TMEM lane)
-        float kscale = 1.f;
-        if constexpr (C::FP8) {
-          kscale = ks_ring[0];
-#pragma unroll
-          for (int i = 0; i + 1 < PF; ++i) ks_ring[i] = ks_ring[i + 1];
-          ks_ring[PF - 1] = load_scale(kt + PF);
-        }
-        for (int g = 0; g < groups; ++g, ++acc_iter) {
-          if (C::EG > 1 && static_cast<int>(acc_iter % C::EG) != grp) continue;   // another group's
-          const int b = acc_iter % C::NBUF;
-          if (!DSA_TIMED(3, mbar_wait<C::EPI_SLEEP>(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag))) { ok = false; break; }
-#ifdef DSA_PIPE_STATS
-          const long long tc0_ = clock64();
-#endif
-          tc_fence_after();
-          const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::ACC_COLS;
-          const int j_lo = g * C::TPA;
-          const int j_hi = min(j_lo + C::TPA, wi.n_tok);
-          if constexpr (C::ONE_QUERY_PER_WARP) {
-            const int j = part;                                        // this warp's query
-            if (j < wi.n_tok && key0 <= last_key(j)) {                 // warp-uniform
-              float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-#if DSA_TMEM_X64
-              uint32_t r[64];
-              tmem_ld_32x32b_x64(tbase + j * 64, r);
-              tmem_ld_wait();
-              relu_wsum32_reg(*reinterpret_cast<uint32_t(*)[32]>(r), wr_lo, a0, a1);
-              relu_wsum32_reg(*reinterpret_cast<uint32_t(*)[32]>(r + 32), wr_hi, a0, a1);
-#else
-              uint32_t r0[32], r1[32];
-              tmem_ld_32x32b_x32(tbase + j * 64, r0);
-              tmem_ld_32x32b_x32(tbase + j * 64 + 32, r1);
-              tmem_ld_wait();
-              relu_wsum32_reg(r0, wr_lo, a0, a1);
-              relu_wsum32_reg(r1, wr_hi, a0, a1);
-#endif
-              const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
-              const bool valid = key <= last_key(j);
-              if (valid) args.scores[rowoff[j] + key] = v;
-              if (C::HIST && args.row_hist) hist_count(j, v, valid);
-            }
-          } else if constexpr (C::H >= 32 && C::CHUNKED) {
-            // many epilogue warps: one 32-column chunk in registers at a time
-            constexpr int CPT = C::H / 32;
-            for (int j = j_lo + part; j < j_hi; j += SPLIT) {
-              if (key0 > last_key(j)) continue;                        // the tile is after this query
-              float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-#pragma unroll
-              for (int c = 0; c < CPT; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tbase + (j - j_lo) * C::H + c * 32, r);
-                tmem_ld_wait();
-                relu_wsum32(r, wq + j * C::H + c * 32, a0, a1);
-              }
-              const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
-              const bool valid = key <= last_key(j);
-              if (valid) args.scores[rowoff[j] + key] = v;
-              if (C::HIST && args.row_hist) hist_count(j, v, valid);
-            }
-          } else if constexpr (C::H >= 32) {
-            // QB queries per pass: their loads are in flight behind one tcgen05.wait::ld
-            constexpr int CPT = C::H / 32;
-            for (int j0 = j_lo + part; j0 < j_hi; j0 += C::QB * SPLIT) {
-              uint32_t r[C::QB][CPT][32];
-              bool live[C::QB];
-              bool any = false;
-#pragma unroll
-              for (int u = 0; u < C::QB; ++u) {
-                const int j = j0 + u * SPLIT;
-                live[u] = j < j_hi && key0 <= last_key(j);             // warp-uniform
-                any |= live[u];
-                if (live[u]) {
-#pragma unroll
-                  for (int c = 0; c < CPT; ++c) tmem_ld_32x32b_x32(tbase + (j - j_lo) * C::H + c * 32, r[u][c]);
-                }
-              }
-              if (!any) continue;                                      // the tile is after these queries
-              tmem_ld_wait();
-#pragma unroll
-              for (int u = 0; u < C::QB; ++u) {
-                const int j = j0 + u * SPLIT;
-                if (live[u]) {
-                  const float v = relu_wsum<CPT>(r[u], wq + j * C::H) * kscale;
-                  const bool valid = key <= last_key(j);
-                  if (valid) args.scores[rowoff[j] + key] = v;
-                  if (C::HIST && args.row_hist) hist_count(j, v, valid);
-                }
-              }
-            }
-          } else {
-            // H < 32: one 32-column load holds 32/H queries
-            constexpr int QPC = 32 / C::H;
-            for (int c = part; c < C::N / 32; c += SPLIT) {
-              const int jc = j_lo + c * QPC;
-              if (jc >= j_hi) break;
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(tbase + c * 32, r);
-              tmem_ld_wait();
-#pragma unroll
-              for (int u = 0; u < QPC; ++u) {
-                const int j = jc + u;
-                if (j < j_hi) {
-                  float acc = 0.f;
-#pragma unroll
-                  for (int h = 0; h < C::H; ++h)
-                    acc = fmaf(wq[j * C::H + h], fmaxf(__uint_as_float(r[u * C::H + h]), 0.f), acc);
-                  const float v = acc * kscale;
-                  const bool valid = key <= last_key(j);
-                  if (valid) args.scores[rowoff[j] + key] = v;
-                  if (C::HIST && args.row_hist) hist_count(j, v, valid);
-                }
-              }
-            }
+      // the tile loop, compiled twice: plain causal limits (one add per query) and limits
+      // over a compressed cache (a division), so the plain loop carries no compression test
+      auto tile_loop = [&](auto compressed) {
+        constexpr bool kCompressed = decltype(compressed)::value;
+        auto last_key = [&](int j) -> int {
+          if constexpr (kCompressed) return (wi.pos0 + j + 1) / cmp - 1;
+          else return wi.pos0 + j;
+        };
+        for (int kt = wi.kt_begin; kt < wi.kt_end && ok; ++kt) {
+          const int key0 = kt * C::BM;                      // first key of the tile
+          const int key = key0 + sub * 32 + lane;           // this thread's key (its TMEM lane)
+          float kscale = 1.f;
+          if constexpr (C::FP8) {
+            kscale = ks_ring[0];
+  #pragma unroll
+            for (int i = 0; i + 1 < PF; ++i) ks_ring[i] = ks_ring[i + 1];
+            ks_ring[PF - 1] = load_scale(kt + PF);
           }
-          tc_fence_before();
-          __syncwarp();
-#ifdef DSA_PIPE_STATS
-          st_[4] += clock64() - tc0_;
-#endif
-          if (lane == 0) mbar_arrive(&acc_empty[b]);
+          for (int g = 0; g < groups; ++g, ++acc_iter) {
+            if (C::EG > 1 && static_cast<int>(acc_iter % C::EG) != grp) continue;   // another group's
+            const int b = acc_iter % C::NBUF;
+            if (!DSA_TIMED(3, mbar_wait<C::EPI_SLEEP>(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag))) { ok = false; break; }
+  #ifdef DSA_PIPE_STATS
+            const long long tc0_ = clock64();
+  #endif
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::ACC_COLS;
+            const int j_lo = g * C::TPA;
+            const int j_hi = min(j_lo + C::TPA, wi.n_tok);
+            if constexpr (C::ONE_QUERY_PER_WARP) {
+              const int j = part;                                        // this warp's query
+              if (j < wi.n_tok && key0 <= last_key(j)) {                 // warp-uniform
+                float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+  #if DSA_TMEM_X64
+                uint32_t r[64];
+                tmem_ld_32x32b_x64(tbase + j * 64, r);
+                tmem_ld_wait();
+                relu_wsum32_reg(*reinterpret_cast<uint32_t(*)[32]>(r), wr_lo, a0, a1);
+                relu_wsum32_reg(*reinterpret_cast<uint32_t(*)[32]>(r + 32), wr_hi, a0, a1);
+  #else
+                uint32_t r0[32], r1[32];
+                tmem_ld_32x32b_x32(tbase + j * 64, r0);
+                tmem_ld_32x32b_x32(tbase + j * 64 + 32, r1);
+                tmem_ld_wait();
+                relu_wsum32_reg(r0, wr_lo, a0, a1);
+                relu_wsum32_reg(r1, wr_hi, a0, a1);
+  #endif
+                const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+                const bool valid = key <= last_key(j);
+                if (valid) args.scores[rowoff[j] + key] = v;
+                if (C::HIST && args.row_hist) hist_count(j, v, valid);
+              }
+            } else if constexpr (C::H >= 32 && C::CHUNKED) {
+              // many epilogue warps: one 32-column chunk in registers at a time
+              constexpr int CPT = C::H / 32;
+              for (int j = j_lo + part; j < j_hi; j += SPLIT) {
+                if (key0 > last_key(j)) continue;                        // the tile is after this query
+                float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+  #pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                  uint32_t r[32];
+                  tmem_ld_32x32b_x32(tbase + (j - j_lo) * C::H + c * 32, r);
+                  tmem_ld_wait();
+                  relu_wsum32(r, wq + j * C::H + c * 32, a0, a1);
+                }
+                const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+                const bool valid = key <= last_key(j);
+                if (valid) args.scores[rowoff[j] + key] = v;
+                if (C::HIST && args.row_hist) hist_count(j, v, valid);
+              }
+            } else if constexpr (C::H >= 32) {
+              // QB queries per pass: their loads are in flight behind one tcgen05.wait::ld
+              constexpr int CPT = C::H / 32;
+              for (int j0 = j_lo + part; j0 < j_hi; j0 += C::QB * SPLIT) {
+                uint32_t r[C::QB][CPT][32];
+                bool live[C::QB];
+                bool any = false;
+  #pragma unroll
+                for (int u = 0; u < C::QB; ++u) {
+                  const int j = j0 + u * SPLIT;
+                  live[u] = j < j_hi && key0 <= last_key(j);             // warp-uniform
+                  any |= live[u];
+                  if (live[u]) {
+  #pragma unroll
+                    for (int c = 0; c < CPT; ++c) tmem_ld_32x32b_x32(tbase + (j - j_lo) * C::H + c * 32, r[u][c]);
+                  }
+                }
+                if (!any) continue;                                      // the tile is after these queries
+                tmem_ld_wait();
+  #pragma unroll
+                for (int u = 0; u < C::QB; ++u) {
+                  const int j = j0 + u * SPLIT;
+                  if (live[u]) {
+                    const float v = relu_wsum<CPT>(r[u], wq + j * C::H) * kscale;
+                    const bool valid = key <= last_key(j);
+                    if (valid) args.scores[rowoff[j] + key] = v;
+                    if (C::HIST && args.row_hist) hist_count(j, v, valid);
+                  }
+                }
+              }
+            } else {
+              // H < 32: one 32-column load holds 32/H queries
+              constexpr int QPC = 32 / C::H;
+              for (int c = part; c < C::N / 32; c += SPLIT) {
+                const int jc = j_lo + c * QPC;
+                if (jc >= j_hi) break;
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tbase + c * 32, r);
+                tmem_ld_wait();
+  #pragma unroll
+                for (int u = 0; u < QPC; ++u) {
+                  const int j = jc + u;
+                  if (j < j_hi) {
+                    float acc = 0.f;
+  #pragma unroll
+                    for (int h = 0; h < C::H; ++h)
+                      acc = fmaf(wq[j * C::H + h], fmaxf(__uint_as_float(r[u * C::H + h]), 0.f), acc);
+                    const float v = acc * kscale;
+                    const bool valid = key <= last_key(j);
+                    if (valid) args.scores[rowoff[j] + key] = v;
+                    if (C::HIST && args.row_hist) hist_count(j, v, valid);
+                  }
+                }
+              }
+            }
+            tc_fence_before();
+            __syncwarp();
+  #ifdef DSA_PIPE_STATS
+            st_[4] += clock64() - tc0_;
+  #endif
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+          }
         }
-      }
+      };
+      if (cmp == 1)
+        tile_loop(std::false_type{});
+      else
+        tile_loop(std::true_type{});
     }
   }
 
