@@ -1,25 +1,33 @@
 #!/usr/bin/env python
 """Indexer throughput on B200: query-key pairs scored and selected per second.
 
-A step is one pass of the whole hot path over the decode-batch workload
-(32 sequences x 32768 cached keys, H_I=64, d_I=128, bf16, top_k=2048, one query per
-sequence): append the step's new keys to the cache, score every (query, key) pair
-(tensor-core logits + fused ReLU / head-weighted sum), select the top 2048 per
-query.  Steps are captured in a CUDA graph and replayed; the K cache (268 MB) is
-larger than L2, so no flush is needed between steps.
+A step is one pass of the whole hot path over one batch of a workload: append the step's
+new keys to the indexer K cache (quantising them for an FP8 cache), quantise the queries
+(FP8), score every causal (query, key) pair (tensor-core logits with the fused ReLU /
+head-weighted sum / causal mask) and select the top 2048 keys per query.
+
+The headline line is the long FP8 prefill (1 sequence of 65536 tokens, H_I=64, d_I=128,
+E4M3 with a per-token scale, top_k=2048), the largest single-GPU workload.  The line's
+"configs" block carries the same measurement for the decode batch (32 x 32768 keys, bf16),
+the bf16 prefill (L=16384) and the ragged FP8 decode (16 sequences of 4096..131072 keys,
+2 queries each), each with its own roofline, e2e and CPU-oracle baseline.  Steps are
+captured in CUDA graphs and replayed; every workload's inputs exceed the 126 MB L2, so no
+flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Under torchrun every rank processes its own 32 sequences (weak scaling, no
-collective on the data path); the time is the max over ranks and `value` counts
-the pairs of all ranks.  `--impl reference` times the fp64 CPU oracle on a
-bounded sample of the same workload.
+Under torchrun every rank processes its own copy-shaped workload (its own seed: weak
+scaling, no collective on the data path); the time is the max over ranks and `value`
+counts the pairs of all ranks.  `--impl reference` times the fp64 CPU oracle on a bounded
+sample of the headline workload.
 """
 
 from __future__ import annotations
 
 import argparse
+import contextlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -41,21 +49,27 @@ WORKLOADS = {
     "decode8": "ragged decode FP8: 16 seqs, lengths U[4096,131072], 2 queries/seq, H_I=64, d_I=128, top_k=2048",
     "tiny": "tiny prefill: 1 seq L=512, H_I=4, d_I=64, bf16, top_k=32",
 }
-WORKLOAD = WORKLOADS["decode"]
+HEADLINE = "prefill8"                       # the largest single-GPU workload
+SUBCONFIGS = ("decode", "prefill", "decode8")
+# steps captured per CUDA graph: short decode steps are batched, long prefill steps go one by one
+GRAPH_STEPS = {"decode": 50, "decode8": 50, "prefill": 1, "prefill8": 1, "tiny": 50}
+E2E_STEPS = {"decode": 200, "decode8": 200, "prefill": 20, "prefill8": 10, "tiny": 50}
+MIN_TIMED_S = 1.0                           # sub-configurations time at least this long
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40, help="timed steps of the headline workload")
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--graph-steps", type=int, default=50, help="steps captured per CUDA graph")
-    ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work for the oracle baseline")
+    ap.add_argument("--kernel-samples", type=int, default=12,
+                    help="graph replays whose profiled step gives the median kernel times")
+    ap.add_argument("--cpu-seconds", type=float, default=4.0, help="oracle CPU work per workload for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode", "prefill", "prefill8", "decode8", "tiny"], default="decode",
-                    help="decode (the default) is the measured workload; the others are for profiling")
+    ap.add_argument("--no-side", action="store_true", help="skip the after-selection / RoPE / compressed sections")
+    ap.add_argument("--workload", choices=["all", "decode", "prefill", "prefill8", "decode8", "tiny"], default="all",
+                    help="all (the default): the headline plus the per-config blocks; one name: that workload alone")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="profiling only: run a prefill workload at this sequence length instead")
     ap.add_argument("--profile-steps", type=int, default=0,
@@ -88,7 +102,7 @@ def job_value(pairs_per_rank: int, world: int, ms_per_step: float) -> float:
 
 # ----------------------------------------------------------------------------- workload
 
-def workload(rank: int, name: str = "decode"):
+def workload(rank: int, name: str):
     """The workload each rank processes; ranks draw different seeds (weak scaling)."""
     from sparse_attention_token_02_b200 import workloads as W
     make = {"decode": W.decode, "prefill": W.prefill, "prefill8": W.prefill8, "decode8": W.decode8,
@@ -102,9 +116,20 @@ def host_inputs(wl):
     return W.make_inputs(wl)
 
 
-# ----------------------------------------------------------------------------- oracle timing
+# ----------------------------------------------------------------------------- oracle timing (CPU baseline)
 
-def _oracle_cores():
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
         return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -112,77 +137,174 @@ def _oracle_cores():
         return os.cpu_count() or 1
 
 
-def _oracle_row(wl, inp, b, n_keys):
-    """One decode row of sequence b restricted to its first n_keys keys, through the oracle."""
-    import oracle
-    kv = oracle.bf16_bits_to_f64(inp["k_bits"][b][:n_keys])
-    qv = oracle.bf16_bits_to_f64(inp["q_bits"][b: b + 1])
-    res = oracle.decode_oracle(qv, [kv], inp["w"][b: b + 1].astype(np.float64), [n_keys], 1, wl.top_k)
-    assert res["idx"].shape == (1, wl.top_k)
-    return n_keys
+class OracleRows:
+    """The oracle's work for one query row of a workload, as a step does it per token: for an
+    FP8 cache, quantise the token's own key row (the append) and its query (the oracle's
+    codec); then score the query against keys 0..p and take the top-k.
+
+    The history keys the scores read are inputs, already in the cache when a step runs; for
+    the timing they are the bf16 source values decoded to fp64 (the fp64 contraction costs the
+    same whatever the values are), so that a sample of rows does not first have to run the
+    slow reference codec over the whole cache."""
+
+    def __init__(self, wl, inp):
+        import oracle
+        self.oracle, self.wl, self.inp = oracle, wl, inp
+        self.fp8 = wl.dtype == "fp8"
+        self.row_seq = np.repeat(np.arange(wl.num_seqs), wl.q_lens)
+        self.row_pos = np.concatenate([np.arange(L - n, L) for L, n in zip(wl.seq_lens, wl.q_lens)])
+        self._keys = {}
+
+    def keys(self, b):
+        if b not in self._keys:
+            self._keys[b] = self.oracle.bf16_bits_to_f64(self.inp["k_bits"][b])
+        return self._keys[b]
+
+    def prepare(self, r: int):
+        """Everything row r needs that is an input, not oracle work: its sequence's key values,
+        its query bits and head weights (drawn here when the inputs are generated lazily)."""
+        b, p = int(self.row_seq[r]), int(self.row_pos[r])
+        self.keys(b)
+        return self.inp["q_bits"][r], self.inp["w"][r], self.inp["k_bits"][b][p: p + 1]
+
+    def row(self, r: int, n_keys: int | None = None, prepared=None) -> int:
+        """The oracle on packed row r (its first n_keys keys if given); returns the pairs scored."""
+        o = self.oracle
+        b, p = int(self.row_seq[r]), int(self.row_pos[r])
+        n = p + 1 if n_keys is None else min(p + 1, n_keys)
+        bits, w, kbits = prepared if prepared is not None else self.prepare(r)
+        if self.fp8:
+            o.quantize_rows(o.bf16_bits_to_f64(kbits).astype(np.float32))          # the token's key (append)
+            codes, sc = o.quantize_rows(o.bf16_bits_to_f64(bits.reshape(1, -1)).astype(np.float32))
+            qv = (o.e4m3_decode(codes) * np.float64(sc[0])).reshape(bits.shape)
+        else:
+            qv = o.bf16_bits_to_f64(bits)
+        s = o.row_scores(qv, self.keys(b)[:n], np.asarray(w, dtype=np.float64))
+        o.topk_row(s, self.wl.top_k)
+        return n
 
 
-def oracle_sample(wl, inp, seconds: float):
-    """Times the fp64 oracle on whole decode rows of this workload until `seconds` pass."""
-    pairs = rows = b = 0
-    t0 = time.perf_counter()
-    while True:
-        pairs += _oracle_row(wl, inp, b, wl.seq_lens[b])
-        rows += 1
-        b = (b + 1) % wl.num_seqs
-        if time.perf_counter() - t0 >= seconds:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": pairs / dt, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
-            "sample": f"{rows} whole decode rows of {wl.seq_lens[0]} keys (numpy fp64 oracle, {dt:.1f} s)"}
+def oracle_baseline(wl, inp, seconds: float, threads: int | None = None, seed: int = 0) -> dict:
+    """Times the fp64 oracle on whole query rows of the workload, taken in a seeded random
+    order, until `seconds` of oracle time have passed (or every row is done); the rate is the
+    sampled rows' pairs per second, which is the whole workload's rate when the rows are a
+    sample of it ("extrapolated" says so)."""
+    from threadpoolctl import threadpool_limits
+    orc = OracleRows(wl, inp)
+    T = wl.total_q
+    order = np.random.default_rng(seed).permutation(T)
+    busy = pairs = rows = 0
+    limit = threadpool_limits(limits=threads) if threads else contextlib.nullcontext()
+    with limit:
+        cores = _blas_threads()
+        t_prep = 0.0
+        for r in order:
+            t = time.perf_counter()
+            prep = orc.prepare(int(r))                        # inputs: drawn before timing
+            t_prep += time.perf_counter() - t
+            t = time.perf_counter()
+            pairs += orc.row(int(r), prepared=prep)
+            busy += time.perf_counter() - t
+            rows += 1
+            if busy >= seconds or t_prep >= max(30.0, 6 * seconds):   # bounded: the bench must end in minutes
+                break
+    extrapolated = rows < T
+    per_row = ("quantise the token's key and query (oracle codec), scores, top-k" if wl.dtype == "fp8"
+               else "scores, top-k")
+    sample = (f"{rows} of {T} query rows ({'seeded random order, ' if extrapolated else ''}{pairs} pairs, "
+              f"{busy:.1f} s of numpy fp64 oracle; per row: {per_row})")
+    return {"value": pairs / busy, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+            "extrapolated": extrapolated, "model": cpu_model()}
+
+
+def cpu_baselines(name, wl, inp, seconds) -> dict:
+    """cpu_baseline of one workload: the oracle on the host's BLAS threads, plus one thread
+    on the tiny and decode-batch workloads."""
+    out = oracle_baseline(wl, inp, seconds)
+    if name in ("tiny", "decode"):
+        one = oracle_baseline(wl, inp, seconds / 2, threads=1)
+        out["threads_1"] = {"value": one["value"], "sample": one["sample"], "extrapolated": one["extrapolated"]}
+    return out
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step is a bounded sample of the workload
-    (whole rows when the step budget allows, else a row's first keys, at least top_k+1),
-    sized so that warm-up plus all steps take about two and a half minutes."""
+    """The oracle as the reference arm, on the headline workload: each step is a bounded
+    sample of it (a few whole query rows, in a seeded random order), sized so that warm-up
+    plus all steps take about two and a half minutes."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = workload(0)
-    inp = host_inputs(wl)
-    L = wl.seq_lens[0]
+    name = HEADLINE if args.workload == "all" else args.workload
+    wl = workload(0, name)
+    inp = reference_inputs(wl)
+    orc = OracleRows(wl, inp)
+    order = np.random.default_rng(1).permutation(wl.total_q)
+    prep = orc.prepare(int(order[0]))
     t = time.perf_counter()
-    _oracle_row(wl, inp, 0, L)
-    row_s = time.perf_counter() - t
+    orc.row(int(order[0]), prepared=prep)
+    row_s = max(time.perf_counter() - t, 1e-6)
     budget = 150.0 / max(1, args.steps + args.warmup)
-    if budget >= row_s:
-        rows_per_step, keys = max(1, min(wl.num_seqs, int(budget / row_s))), L
-    else:
-        rows_per_step, keys = 1, int(min(L, max(wl.top_k + 1, L * budget / row_s)))
-    secs, pairs = [], 0
-    b = 0
-    for i in range(args.warmup + args.steps):
+    rows_per_step = max(1, min(wl.total_q, int(budget / row_s)))
+    secs, pairs, i = [], 0, 1
+    for s in range(args.warmup + args.steps):
+        rows = [int(order[(i + j) % len(order)]) for j in range(rows_per_step)]
+        i += rows_per_step
+        preps = [orc.prepare(r) for r in rows]             # inputs: drawn before the step's timing
         t = time.perf_counter()
         n = 0
-        for _ in range(rows_per_step):
-            n += _oracle_row(wl, inp, b, keys)
-            b = (b + 1) % wl.num_seqs
-        if i >= args.warmup:
+        for r, pr in zip(rows, preps):
+            n += orc.row(r, prepared=pr)
+        if s >= args.warmup:
             secs.append(time.perf_counter() - t)
             pairs += n
     value = pairs / sum(secs)
-    sample = (f"per step {rows_per_step} decode row(s) x {keys} keys of the workload "
-              f"(numpy fp64 oracle; {len(secs)} steps, {sum(secs):.1f} s)")
-    info = {"value": value, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle", "sample": sample}
+    sample = (f"per step {rows_per_step} whole query row(s) of the workload in a seeded random order "
+              f"(numpy fp64 oracle: scores + top-k; {len(secs)} steps, {sum(secs):.1f} s), "
+              f"extrapolated to the workload by pair count")
+    info = {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle", "sample": sample,
+            "model": cpu_model()}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample},
+            "data": "synthetic", "config": {"workload": WORKLOADS[name], "sample": sample},
             "cpu_baseline": info,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
+def reference_inputs(wl):
+    """Host inputs of a workload; for the long prefill only the key rows and the query / weight
+    rows the reference arm can reach are drawn (any rows of a tensor regenerate alone)."""
+    from sparse_attention_token_02_b200 import workloads as W
+    if wl.total_q <= 20000:
+        return W.make_inputs(wl)
+
+    n = W.CHUNK_ROWS
+    T = wl.total_q
+    return {"k_bits": [W.f32_to_bf16_bits(W.key_rows(wl, b)) for b in range(wl.num_seqs)],
+            "q_bits": _ChunkRows(lambda c: W.f32_to_bf16_bits(W.query_rows(wl, c * n, min(T, (c + 1) * n))), n),
+            "w": _ChunkRows(lambda c: W.weight_rows(wl, c * n, min(T, (c + 1) * n)), n)}
+
+
+class _ChunkRows:
+    """Rows of a generated tensor, drawn a chunk of rows at a time on first use."""
+
+    def __init__(self, fn, rows_per_chunk):
+        self.fn, self.n, self.cache = fn, rows_per_chunk, {}
+
+    def __getitem__(self, r):
+        c, i = divmod(int(r), self.n)
+        if c not in self.cache:
+            self.cache[c] = self.fn(c)
+        return self.cache[c][i]
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """nvidia-smi samples (every 200 ms) over the whole run; summary() gives the samples of
+    one timed region by wall-clock time."""
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -205,20 +327,26 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self, t_begin: float, t_end: float):
-        """Summary of the samples taken between the wall-clock times t_begin and t_end."""
+    def close(self):
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=2)
+        self.proc = None
+
+    def summary(self, t_begin: float, t_end: float):
+        """Median SM clock, max clock and active throttle reasons of the samples taken between
+        the wall-clock times t_begin and t_end."""
+        if not self.lines and self.proc is None:
+            return None
         import datetime
-        sm, mx, reasons, n_all = [], None, set(), 0
+        sm, mx, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in list(self.lines):
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 10:
                 continue
@@ -227,19 +355,23 @@ class ClockSampler:
                 clk, mx = float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            n_all += 1
             if not (t_begin - 0.1 <= ts <= t_end + 0.1):
                 continue
             sm.append(clk)
+            try:
+                power.append(float(parts[4]))
+            except ValueError:
+                pass
             for n, v in zip(names, parts[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0, "samples_total": n_all}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
 
 
-# ----------------------------------------------------------------------------- our path
+# ----------------------------------------------------------------------------- roofline denominators
 
 def peaks():
     """Roofline denominators: the measured copy bandwidth and cuBLAS bf16 GEMM
@@ -254,11 +386,16 @@ def peaks():
             "kind": kind}
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the decode logits kernel from the committed ncu summary,
-    or None when the kernel source changed since those counters were taken."""
+PROFILE_NAMES = {"decode": "decode_bf16", "prefill": "prefill_bf16", "prefill8": "prefill_fp8",
+                 "decode8": "decode8_fp8", "tiny": "tiny_bf16"}
+
+
+def profiled_traffic(name: str):
+    """DRAM bytes per launch of a workload's logits kernel from the committed ncu summary
+    profiles/logits_<workload>_traffic.md, or None when there is none or the kernel source
+    changed since those counters were taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "logits_decode_bf16_traffic.md")
+    path = os.path.join(ROOT, "profiles", f"logits_{PROFILE_NAMES[name]}_traffic.md")
     src = os.path.join(ROOT, "sparse_attention_token_02_b200", "csrc", "kernels_logits.cu")
     try:
         text = open(path).read()
@@ -270,6 +407,8 @@ def profiled_traffic():
     except Exception:
         return None
 
+
+# ----------------------------------------------------------------------------- side measurements
 
 # Before a launch timed alone, the GPU spins this many cycles (about 150 us) after the L2
 # flush, so the host has enqueued the start event, the launch and the end event before the
@@ -448,6 +587,8 @@ def compressed_prefill_timing(api, stream, dev, m=4, reps=5, L=16384, H=64, d=12
             "tflops": flops / (ms * 1e-3) / 1e12, "note": "logits + top-k, causal over complete blocks"}
 
 
+# ----------------------------------------------------------------------------- our path
+
 class Harness:
     """Device state and one step of the hot path for a workload.
 
@@ -527,40 +668,12 @@ class Harness:
         return 2.0 * self.wl.pairs * self.wl.H * self.wl.d
 
 
-def run_ours(args):
+def measure(name, hx, args, steps, world, dist, clocks, wl, inp, rank):
+    """One workload's block: device-timed steps in CUDA graphs, median kernel times,
+    roofline of the logits kernel, end-to-end steps from pinned host memory, CPU baseline."""
     import torch
-    import torch.distributed as dist
-
-    from sparse_attention_token_02_b200 import api
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    stream = torch.cuda.Stream(device=dev)
-
-    wl = workload(rank, args.workload)
-    if args.seq_len and wl.kind == "prefill":
-        from sparse_attention_token_02_b200 import workloads as W
-        wl = W.scaled(wl, seq_lens=(args.seq_len,), q_lens=(args.seq_len,))
-    inp = host_inputs(wl)
-    hx = Harness(wl, inp, dev, stream)
-
-    if args.profile_steps > 0:
-        with torch.cuda.stream(stream):
-            for _ in range(args.profile_steps):
-                hx.step()
-        api.dsa_check_device_errors(stream)
-        if world > 1:
-            dist.destroy_process_group()
-        return 0
+    api, stream, dev = hx.api, hx.stream, hx.dev
+    G = GRAPH_STEPS[name]
 
     # uncaptured warm-up (also plans the batch once)
     with torch.cuda.stream(stream):
@@ -570,7 +683,6 @@ def run_ours(args):
 
     # capture G steps; the middle one carries kernel-timing events (events between kernels
     # would keep the next kernel from starting its prologue early, so the other steps have none)
-    G = max(1, min(args.graph_steps, args.steps))
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     with torch.cuda.stream(stream):
         for e in ev:
@@ -585,21 +697,27 @@ def run_ours(args):
             hx.step()
             api.dsa_set_profile_events(None, None, None)
     launches_per_step = (api.dsa_kernel_launch_count() - n0) / G
-    replays = max(1, args.steps // G)
-    K = replays * G
     with torch.cuda.stream(stream):
         graph.replay()
     stream.synchronize()
     api.dsa_check_device_errors(stream)
 
+    if steps is None:
+        # sub-configurations: at least MIN_TIMED_S of timed work, a whole number of graphs
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            graph.replay()
+            t1.record(stream)
+        stream.synchronize()
+        est = t0.elapsed_time(t1) / G
+        steps = max(args.steps, int(math.ceil(MIN_TIMED_S * 1e3 / max(est, 1e-3))))
+        steps = max(steps, G)
+        steps = int(max_over_ranks(steps, dist if world > 1 else None))   # every rank replays the same count
+    replays = int(math.ceil(steps / G))
+    K = replays * G
+
     # timed region
-    uuid = None
-    try:
-        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        pass
-    clocks = ClockSampler(uuid)
-    time.sleep(0.5)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -614,31 +732,78 @@ def run_ours(args):
     wall1 = time.time()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop(wall0, wall1)
-    ms_total = t0.elapsed_time(t1)
-    # kernel times of the profiled step of the last replay in the timed region
-    logits_ms = ev[0].elapsed_time(ev[1])
-    topk_ms = ev[1].elapsed_time(ev[2])
-    api.dsa_check_device_errors(stream)
-    ms_total = max_over_ranks(ms_total, dist if world > 1 else None)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), dist if world > 1 else None)
     ms_step = ms_total / K
-    pairs_step = wl.pairs * world
-    value = job_value(wl.pairs, world, ms_step)
+    clk = clocks.summary(wall0, wall1) if clocks is not None else None
 
-    # end to end from pinned host buffers: upload the step's inputs, run, read the result back
+    # kernel times: the profiled step of each of `kernel-samples` further replays
+    lg, tk = [], []
+    for _ in range(max(10, args.kernel_samples)):
+        with torch.cuda.stream(stream):
+            graph.replay()
+        stream.synchronize()
+        lg.append(ev[0].elapsed_time(ev[1]))
+        tk.append(ev[1].elapsed_time(ev[2]))
+    logits_ms, topk_ms = statistics.median(lg), statistics.median(tk)
+    api.dsa_check_device_errors(stream)
+    del graph
+
+    e2e = e2e_block(name, hx, dist, world)
+
+    # roofline of the dominant (logits) kernel
+    pk = peaks()
+    if hx.decode:
+        alg = hx.logits_bytes()
+        achieved = alg / (logits_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "traffic": profiled_traffic(name),
+                "peak_source": f"{pk['kind']} hbm_gbs (copy)", "alg_bytes_per_launch": alg}
+    else:
+        alg = hx.logits_flops()
+        achieved = alg / (logits_ms * 1e-3) / 1e12
+        peak = pk["fp8_sustained"] if hx.fp8 else pk["bf16_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(name),
+                "peak_source": (f"{pk['kind']} bf16_tflops_sustained (the kernel runs inside a long loop)" +
+                                (" x 2, the nominal FP8 / bf16 dense ratio" if hx.fp8 else "")),
+                "alg_flops_per_launch": alg,
+                "frac_of_burst_peak": achieved / (pk["fp8_burst"] if hx.fp8 else pk["bf16_burst"])}
+    roof.update({"kernel": f"logits ({wl.kind}, {wl.dtype})", "kernel_ms": logits_ms,
+                 "kernel_ms_samples": len(lg), "kernel_ms_spread": [min(lg), max(lg)]})
+    step_bytes = hx.logits_bytes()
+    block = {
+        "workload": WORKLOADS[name], "pairs_per_step_per_gpu": wl.pairs, "steps": K, "graph_steps": G,
+        "ms_per_step": ms_step, "value": job_value(wl.pairs, world, ms_step), "unit": UNIT,
+        "dtype": "fp8_e4m3" if hx.fp8 else "bf16",
+        "step": ("kcache_append + " + ("quantise q + " if hx.fp8 else "") +
+                 ("decode" if hx.decode else "prefill") + " (logits + top-k)"),
+        "roofline": roof,
+        "kernels_ms": {"logits": logits_ms, "topk": topk_ms, "samples": len(lg)},
+        "step_frac_of_hbm": (step_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm"]) if hx.decode else None,
+        "e2e": e2e,
+        "gpu_launches": int(round(launches_per_step * K)),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        block["cpu_baseline"] = cpu_baselines(name, wl, inp, args.cpu_seconds)
+    else:
+        block["cpu_baseline"] = None
+    return block
+
+
+def e2e_block(name, hx, dist, world):
+    """End to end from pinned host memory: every step uploads its inputs and reads its
+    selection back.  Decode goes through the library's one-call host step
+    (dsa_indexer_decode_host with a completion event: the read-back of a step overlaps the
+    kernels of the next); prefill copies around the device calls.  Steps are enqueued back
+    to back; the events bracket all of them, the end event after the last read-back."""
+    import torch
+    api, stream, dev = hx.api, hx.stream, hx.dev
     k_h, q_h, w_h = hx.k_step_host.pin_memory(), hx.q_src_host.pin_memory(), hx.w_host.pin_memory()
     k_d, q_d, w_d = torch.empty_like(hx.k_step), torch.empty_like(hx.q_src), torch.empty_like(hx.w)
     oi_h = torch.empty(hx.out_idx.shape, dtype=torch.int32, pin_memory=True)
     os_h = torch.empty(hx.out_score.shape, dtype=torch.float32, pin_memory=True)
-
     rows_h = hx.rows_host.pin_memory()
-
-    # Each step uploads its inputs from pinned host memory and reads its selection back.
-    # Decode goes through the library's one-call host step (dsa_indexer_decode_host with a
-    # completion event: the read-back of a step overlaps the kernels of the next); prefill
-    # copies around the device call.  Steps are enqueued back to back (the host does not wait
-    # for each one); the events below bracket all of them, the end event placed after the
-    # last step's read-back has completed.
     done = [torch.cuda.Event(), torch.cuda.Event()]
     last = [None]
     batch = api.host_batch(hx.seq_lens, hx.q_lens, hx.k_base)   # built once, like a serving loop's metadata
@@ -661,7 +826,7 @@ def run_ours(args):
     for _ in range(3):
         e2e_step()
     torch.cuda.synchronize(dev)
-    E = max(1, args.e2e_steps if hx.decode else min(args.e2e_steps, 10))
+    E = E2E_STEPS[name]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -680,64 +845,105 @@ def run_ours(args):
     api.dsa_check_device_errors(stream)
     h2d = sum(t.numel() * t.element_size() for t in (k_h, q_h, w_h)) + (rows_h.numel() * 8 if hx.decode else 0)
     d2h = sum(t.numel() * t.element_size() for t in (oi_h, os_h))
+    pairs = hx.wl.pairs * world
+    return {"value": pairs / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": e2e_ms, "steps": E, "host_enqueue_us_per_step": host_us,
+            "path": ("dsa_indexer_decode_host (one C-ABI call per step, library copy streams)" if hx.decode else
+                     "pinned host -> device copies, append / quantise / prefill C-ABI calls, device -> host copies, "
+                     "all on the compute stream")}
 
-    # the selection's consumers (outside the timed step): the latent-row gather the sparse
-    # attention makes and the sorted order, each launch timed alone after an L2 flush
-    after = after_select_timings(api, hx, stream, dev) if hx.decode else None
-    rope = rope_timings(api, stream, dev) if hx.decode else None
-    comp = compressed_timings(api, hx, stream, dev) if hx.decode and not hx.fp8 else None
 
-    # roofline of the dominant kernel (the logits kernel)
-    pk = peaks()
-    if hx.decode:
-        alg = hx.logits_bytes()
-        achieved = alg / (logits_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "traffic": profiled_traffic() if args.workload == "decode" else None,
-                "peak_source": f"{pk['kind']} hbm_gbs", "alg_bytes_per_launch": alg}
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_attention_token_02_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
     else:
-        alg = hx.logits_flops()
-        achieved = alg / (logits_ms * 1e-3) / 1e12
-        peak = pk["fp8_sustained"] if hx.fp8 else pk["bf16_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
-                "peak_source": (f"{pk['kind']} bf16_tflops_sustained" + (" x 2 (FP8/bf16 nominal ratio)" if hx.fp8 else "")),
-                "alg_flops_per_launch": alg,
-                "frac_of_burst_peak": achieved / (pk["fp8_burst"] if hx.fp8 else pk["bf16_burst"])}
-    roof.update({"kernel": f"logits ({wl.kind}, {wl.dtype})", "kernel_ms": logits_ms})
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream(device=dev)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "decode":
-        cpu = oracle_sample(wl, inp, args.cpu_seconds)
+    head = HEADLINE if args.workload == "all" else args.workload
+
+    if args.profile_steps > 0:
+        wl = workload(rank, head)
+        if args.seq_len and wl.kind == "prefill":
+            from sparse_attention_token_02_b200 import workloads as W
+            wl = W.scaled(wl, seq_lens=(args.seq_len,), q_lens=(args.seq_len,))
+        hx = Harness(wl, host_inputs(wl), dev, stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.profile_steps):
+                hx.step()
+        api.dsa_check_device_errors(stream)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    time.sleep(0.5)
+
+    names = [head] + (list(SUBCONFIGS) if args.workload == "all" else [])
+    blocks, side = {}, {}
+    for name in names:
+        wl = workload(rank, name)
+        inp = host_inputs(wl)
+        hx = Harness(wl, inp, dev, stream)
+        blocks[name] = measure(name, hx, args, args.steps if name == head else None, world, dist, clocks, wl,
+                               inp, rank)
+        if name == "decode" and not args.no_side:
+            # the selection's consumers and the fused RoPE / compressed-cache calls (outside the
+            # timed steps), each launch timed alone after an L2 flush
+            side["after_select"] = after_select_timings(api, hx, stream, dev)
+            side["rope_fused"] = rope_timings(api, stream, dev)
+            side["compressed_decode"] = compressed_timings(api, hx, stream, dev)
+        del hx, inp
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+    clocks.close()
+    if args.workload == "all" and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl = workload(0, "tiny")
+        tiny_cpu = cpu_baselines("tiny", wl, host_inputs(wl), args.cpu_seconds)
+    else:
+        tiny_cpu = None
 
     if world > 1:
         dist.barrier()
     if rank == 0:
+        hb = blocks[head]
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8_e4m3" if hx.fp8 else "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.workload], "pairs_per_step_per_gpu": wl.pairs,
+            "metric": METRIC, "value": hb["value"], "unit": UNIT, "n_gpus": world, "steps": hb["steps"],
+            "warmup": args.warmup, "ms_per_step": hb["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": hb["dtype"], "data": "synthetic",
+            "config": {"workload": WORKLOADS[head], "pairs_per_step_per_gpu": hb["pairs_per_step_per_gpu"],
                        "l2": "inputs larger than L2 (126 MB), no flush",
-                       "step": ("kcache_append + " + ("quantise q + " if hx.fp8 else "") +
-                                ("decode" if hx.decode else "prefill") + " (logits + top-k), CUDA graph of %d steps" % G),
-                       "parallelism": f"{world} independent ranks (sequences sharded)"},
-            "roofline": roof,
-            "kernels_ms": {"logits": logits_ms, "topk": topk_ms},
-            "cpu_baseline": cpu,
-            "e2e": {"value": pairs_step / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "host_enqueue_us_per_step": host_us},
-            "gpu_launches": int(round(launches_per_step * K)),
-            "clocks": clk,
+                       "step": hb["step"] + f", CUDA graphs of {hb['graph_steps']} step(s)",
+                       "parallelism": f"{world} independent ranks (each its own workload: weak scaling)"},
+            "roofline": hb["roofline"],
+            "kernels_ms": hb["kernels_ms"],
+            "cpu_baseline": hb["cpu_baseline"],
+            "e2e": hb["e2e"],
+            "gpu_launches": hb["gpu_launches"],
+            "clocks": hb["clocks"],
+            "configs": {n: b for n, b in blocks.items() if n != head},
         }
-        if after is not None:
-            line["after_select"] = after
-        if rope is not None:
-            line["rope_fused"] = rope
-        if comp is not None:
-            line["compressed_decode"] = comp
+        if tiny_cpu is not None:
+            line["tiny_cpu_baseline"] = tiny_cpu
+        line.update(side)
         print(json.dumps(line), flush=True)
-    del graph
     if world > 1:
         dist.destroy_process_group()
     return 0

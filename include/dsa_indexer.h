@@ -215,24 +215,35 @@ DSA_API dsa_status_t dsa_indexer_scores(const dsa_query_t* q, const dsa_kcache_t
  * Decode that allocates no device memory.  (The pages have no counterpart: this
  * is a library entry point for callers that may not allocate.)
  *
- * Same arguments and result as dsa_indexer_decode, for callers that must not
- * allocate device memory at all: a server whose device memory belongs to its own
- * pool, code under a device-memory budget enforced outside CUDA, or a host that
- * forbids allocator calls on its hot path.  dsa_indexer_decode grows a workspace
- * with cudaMalloc; this call instead keeps the score rows and the scheduling tables
- * in one static 16 MiB __device__ array inside the library, which every GPU that
- * loads the library holds until the process exits.  It calls no cudaMalloc,
- * cudaFree or other allocating routine.
- *   fault  optional device int32[2]: zeroed by the call, then receives the first
- *          device fault (code, info) as dsa_check_device_errors would report it;
- *          with NULL, faults are kept in the static array and not reported.
- * Limits: the batch must fit the array: 4 bytes per cached key of every query
- * (rounded up to 4 keys per query) plus its tables, else DSA_ERR_INVALID_ARG says
- * how much it needs.  Every call shares the one array (per device) and leaves its
- * contents behind, so calls that overlap on the GPU (other streams, other host
- * threads) race; serialise them.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.
+ * The decode step for callers that must not allocate device memory at all: a server
+ * whose device memory belongs to its own pool (an allocation behind the pool's back can
+ * fail or fragment it), code under a device-memory budget enforced outside CUDA, or a host
+ * that forbids allocator calls on its hot path.  dsa_indexer_decode grows a workspace with
+ * cudaMalloc; this call instead keeps the score rows and the scheduling tables in one
+ * static 16 MiB __device__ array inside the library, which every GPU that loads the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine, and stages nothing through host memory: its tables reach the array
+ * inside kernel parameters.
+ *
+ * Arguments as for dsa_indexer_decode, with these differences:
+ *   fault      optional device int32[2]: cleared by the call, then receives the first
+ *              device fault (code, info) as dsa_check_device_errors would report it;
+ *              with NULL, faults are kept in the static array and not reported.
+ *   out_score  required (the short-sequence bypass of dsa_indexer_decode is not offered).
+ * The selection is the same (same rule, same tolerance of exact ties at the k-th score);
+ * the route differs: after the logits kernel, one cluster of CTAs per row selects from
+ * the row's scores alone (no coarse histogram from the logits epilogue), so a row may hold
+ * at most 131072 keys (DSA_ERR_UNSUPPORTED beyond).
+ * Limits: the batch must fit the array: 4 bytes per cached key of every query (rounded
+ * up to 4 keys per query) plus its tables, else DSA_ERR_INVALID_ARG says how much it
+ * needs.  Every call shares the one array (per device) and leaves its contents behind, so
+ * calls that overlap on the GPU (other streams, other host threads) race; serialise them.
+ * Set-up: the array is reserved on a device when the library's device code is loaded
+ * there -- with CUDA's lazy module loading (the default) that happens during the first
+ * call on the device, which can therefore fail with a CUDA out-of-memory error on a device
+ * that is already full.  The first call on a device also looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current.  Make one call at
+ * initialisation, before any stream capture.
  */
 DSA_API dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w,
                                                 const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx,

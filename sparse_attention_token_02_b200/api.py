@@ -393,45 +393,3 @@ def dsa_kernel_launch_count() -> int:
 
 def dsa_version() -> str:
     return _lib.load().dsa_version().decode()
-
-
-def dsa_indexer_decode_from_host(q_host, w_host, k_new_host, dst_rows, cache: IndexerKCache, seq_lens, q_lens,
-                                 top_k, q_scale_host=None, k_base=None, dev_bufs=None, stream=None):
-    """A whole decode step from pinned HOST buffers: upload the step's new keys, queries
-    and weights, append the keys, score + select, and copy the result back.
-
-    Returns host (out_idx, out_score).  ``dev_bufs`` (a dict) caches device staging
-    tensors between calls.  The copies are enqueued on the same stream as the kernels.
-    """
-    s = torch.cuda.current_stream() if stream is None else stream
-    dev = cache.k.device
-    bufs = dev_bufs if dev_bufs is not None else {}
-
-    def up(name, t):
-        if t is None:
-            return None
-        d = bufs.get(name)
-        if d is None or d.shape != t.shape or d.dtype != t.dtype:
-            d = torch.empty(t.shape, dtype=t.dtype, device=dev)
-            bufs[name] = d
-        with torch.cuda.stream(s):
-            d.copy_(t, non_blocking=True)
-        return d
-
-    qd, wd, kd, qs = up("q", q_host), up("w", w_host), up("k_new", k_new_host), up("q_scale", q_scale_host)
-    rows = up("dst_rows", dst_rows) if not dst_rows.is_cuda else dst_rows
-    dsa_indexer_kcache_append(cache, kd, rows, stream=s)
-    T = int(np.sum(q_lens))
-    oi = bufs.get("oi")
-    if oi is None or oi.shape != (T, top_k):
-        bufs["oi"] = oi = torch.empty(T, top_k, dtype=torch.int32, device=dev)
-        bufs["os"] = torch.empty(T, top_k, dtype=torch.float32, device=dev)
-        bufs["oi_h"] = torch.empty(T, top_k, dtype=torch.int32, pin_memory=True)
-        bufs["os_h"] = torch.empty(T, top_k, dtype=torch.float32, pin_memory=True)
-    dsa_indexer_decode(qd, cache, wd, seq_lens, q_lens, top_k, q_scale=qs, k_base=k_base, out_idx=oi,
-                       out_score=bufs["os"], stream=s)
-    with torch.cuda.stream(s):
-        bufs["oi_h"].copy_(oi, non_blocking=True)
-        bufs["os_h"].copy_(bufs["os"], non_blocking=True)
-    s.synchronize()
-    return bufs["oi_h"], bufs["os_h"]

@@ -1276,6 +1276,42 @@ dsa_status_t noalloc_scratch(void** out) {
   return DSA_OK;
 }
 
+// The call's scheduling tables travel to the array inside kernel parameters, in chunks of
+// kTableChunk bytes: a parameter block is copied when the launch is enqueued, so the host
+// blob may be freed as soon as the call returns, and nothing is staged through host memory
+// that the driver would have to allocate or pin.
+constexpr int kTableChunk = 16384;
+struct __align__(16) TableChunk {
+  unsigned char bytes[kTableChunk];
+};
+
+// Copies `n` bytes (a multiple of 16) of the chunk to dst; the first chunk of a call also
+// clears the call's two fault words.
+__global__ void __launch_bounds__(256) noalloc_tables_kernel(const __grid_constant__ TableChunk chunk, int n,
+                                                             unsigned char* __restrict__ dst, int* fault_words) {
+  const uint4* src = reinterpret_cast<const uint4*>(chunk.bytes);
+  uint4* out = reinterpret_cast<uint4*>(dst);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n / 16; i += gridDim.x * blockDim.x) out[i] = src[i];
+  if (fault_words != nullptr && blockIdx.x == 0 && threadIdx.x < 2) fault_words[threadIdx.x] = 0;
+}
+
+dsa_status_t noalloc_upload(const std::vector<uint8_t>& blob, unsigned char* dst, int* fault_words,
+                            cudaStream_t stream) {
+  static thread_local TableChunk chunk;
+  size_t off = 0;
+  do {
+    const size_t n = std::min(blob.size() - off, static_cast<size_t>(kTableChunk));
+    if (n) std::memcpy(chunk.bytes, blob.data() + off, n);
+    const int blocks = static_cast<int>((n / 16 + 255) / 256) > 0 ? static_cast<int>((n / 16 + 255) / 256) : 1;
+    noalloc_tables_kernel<<<blocks, 256, 0, stream>>>(chunk, static_cast<int>(n), dst + off,
+                                                      off == 0 ? fault_words : nullptr);
+    DSA_CUDA_TRY(cudaGetLastError(), "table upload kernel launch");
+    ++g_launches;
+    off += n;
+  } while (off < blob.size());
+  return DSA_OK;
+}
+
 }  // namespace
 }  // namespace dsa
 
@@ -1320,12 +1356,10 @@ extern "C" dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const d
   if ((st = noalloc_scratch(&base)) != DSA_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
   int* err = fault ? reinterpret_cast<int*>(fault) : static_cast<int*>(base);
-  DSA_CUDA_TRY(cudaMemsetAsync(err, 0, 2 * sizeof(int), stream), "cudaMemsetAsync(fault words)");
   char* mb = static_cast<char*>(base) + kNoAllocFaultBytes;
   float* d_scores = reinterpret_cast<float*>(mb + align_up(m.total));
-  // the tables come from pageable host memory: the driver stages the copy, nothing is allocated here
-  const std::vector<uint8_t> blob = pack(p, m);
-  DSA_CUDA_TRY(cudaMemcpyAsync(mb, blob.data(), blob.size(), cudaMemcpyHostToDevice, stream), "cudaMemcpyAsync");
+  // the tables (and the cleared fault words) go to the array in kernel parameters
+  if ((st = noalloc_upload(pack(p, m), reinterpret_cast<unsigned char*>(mb), err, stream)) != DSA_OK) return st;
 
   CUtensorMap tk, tq;
   if ((st = encode_rows(&tk, kc->k, fp8, kc->capacity_rows, D, kKeyTile)) != DSA_OK) return st;
@@ -1343,6 +1377,7 @@ extern "C" dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const d
   la.err = err;
   LogitsLaunch L{H, D, fp8, tpa, 1, static_cast<int>(p.cta_items.size()) - 1, stream};
   DSA_CUDA_TRY(launch_logits(L, tk, tq, la), "logits kernel launch");
+  g_launches += L.grid > 0;
   TopkArgs ta{};
   ta.scores = d_scores;
   ta.row_off = la.row_off;
@@ -1357,12 +1392,14 @@ extern "C" dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const d
     s.rows = rows + p.short_first;
     s.n_rows = static_cast<int32_t>(p.short_count);
     DSA_CUDA_TRY(launch_topk_short(s, stream), "top-k (short rows) launch");
+    ++g_launches;
   }
   for (const auto& cl : p.classes) {
     TopkArgs s = ta;
     s.rows = rows + cl.first;
     s.n_rows = static_cast<int32_t>(cl.count);
     DSA_CUDA_TRY(launch_topk(s, cl.ept, cl.cluster, stream), "top-k launch");
+    ++g_launches;
   }
   return DSA_OK;
 }

@@ -94,6 +94,8 @@ def test_compressed_decode_m_1_equals_decode():
             assert abs(a[i] - b[i]) <= 1e-6 * max(abs(a[i]), 1e-30)
         for i in a.keys() ^ b.keys():
             assert abs(a.get(i, b.get(i)) - kth) <= 1e-6 * max(abs(kth), 1e-30)
+    from ._parity import check_rows
+    check_rows(up, b_i, b_s, range(wl.total_q))
 
 
 @pytest.mark.parametrize("dtype,H,d,m", [("bf16", 64, 128, 4), ("fp8", 64, 128, 7), ("bf16", 4, 64, 3)])
@@ -151,9 +153,17 @@ def test_compressed_prefill_m_1_equals_prefill():
     up = Uploaded(wl)
     a_i, a_s = api.dsa_indexer_prefill(up.q, up.cache, up.w, wl.seq_lens, wl.top_k, k_base=up.k_base)
     b_i, b_s = api.dsa_indexer_prefill_compressed(up.q, up.cache, up.w, wl.seq_lens, 1, wl.top_k, k_base=up.k_base)
-    # m = 1 is the same launch sequence: the same selections and scores (the order of a row's
-    # entries is unspecified, so rows are compared sorted by position)
+    # m = 1 is the same launch sequence: the same scores, and the same selections up to exact
+    # ties at the k-th score (which of those are kept is unspecified); both match the oracle
     a_i, a_s, b_i, b_s = (t.cpu().numpy() for t in (a_i, a_s, b_i, b_s))
-    oa, ob = np.argsort(a_i, axis=1), np.argsort(b_i, axis=1)
-    assert np.array_equal(np.take_along_axis(a_i, oa, 1), np.take_along_axis(b_i, ob, 1))
-    assert np.array_equal(np.take_along_axis(a_s, oa, 1), np.take_along_axis(b_s, ob, 1))
+    from ._parity import check_rows
+    rows = list(range(0, wl.total_q, 5)) + [wl.total_q - 1]
+    check_rows(up, b_i, b_s, rows)
+    for r in range(wl.total_q):
+        a = dict(zip(a_i[r].tolist(), a_s[r].tolist()))
+        b = dict(zip(b_i[r].tolist(), b_s[r].tolist()))
+        kth = min(a.values())
+        for i in a.keys() & b.keys():
+            assert a[i] == b[i], f"row {r} index {i}"
+        for i in a.keys() ^ b.keys():
+            assert a.get(i, b.get(i)) == kth, f"row {r}: index {i} selected by one call only, not an exact tie"

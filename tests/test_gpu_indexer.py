@@ -17,7 +17,8 @@ import oracle
 from sparse_attention_token_02_b200 import api
 from sparse_attention_token_02_b200 import workloads as W
 
-from ._parity import RTOL, Uploaded, bits_to_bf16_tensor, check_row
+from ._parity import (RTOL, OracleInputs, Uploaded, bits_to_bf16_tensor, check_row, check_rows, run_indexer,
+                      sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,42 +32,9 @@ def _gpu():
     api.dsa_check_device_errors()
 
 
-def _run(up: Uploaded, decode: bool = False, top_k: int | None = None):
-    wl = up.wl
-    k = wl.top_k if top_k is None else top_k
-    if decode:
-        idx, sc = api.dsa_indexer_decode(up.q, up.cache, up.w, wl.seq_lens, wl.q_lens, k, q_scale=up.q_scale,
-                                         k_base=up.k_base)
-    else:
-        idx, sc = api.dsa_indexer_prefill(up.q, up.cache, up.w, wl.seq_lens, k, q_scale=up.q_scale,
-                                          q_lens=wl.q_lens, k_base=up.k_base)
-    api.dsa_check_device_errors()
-    return idx.cpu().numpy(), sc.cpu().numpy()
-
-
-def _sample_rows(wl: W.Workload, n_mid: int = 8, seed: int = 0):
-    T = wl.total_q
-    rng = np.random.default_rng(seed)
-    picks = {0, 1, T - 1, T - 2}
-    k = wl.top_k
-    seq_pos = []
-    for Lb, n in zip(wl.seq_lens, wl.q_lens):
-        seq_pos += list(range(Lb - n, Lb))
-    seq_pos = np.array(seq_pos)
-    for target in (k - 2, k - 1, k, k + 1, 2 * k + 5):
-        hit = np.nonzero(seq_pos == target)[0]
-        if hit.size:
-            picks.add(int(hit[0]))
-    picks.update(int(x) for x in rng.integers(0, T, size=n_mid))
-    return sorted(p for p in picks if 0 <= p < T)
-
-
-def _check(up: Uploaded, idx, sc, rows, top_k=None):
-    k = up.wl.top_k if top_k is None else top_k
-    rtol = RTOL[up.wl.dtype]
-    orows = up.oracle_rows(rows)
-    for r, orow in zip(rows, orows):
-        check_row(idx[r], sc[r], orow, k, rtol, what=f"{up.wl.name} row {r}")
+_run = run_indexer
+_sample_rows = sample_rows
+_check = check_rows
 
 
 # ----------------------------------------------------------------------------- append / quantise (a1)
@@ -202,7 +170,27 @@ def test_decode_fp8_ragged(q_len):
     _check(up, idx, sc, list(range(wl.total_q)))
 
 
+def _same_set_up_to_exact_ties(idx_a, sc_a, idx_b, sc_b, what):
+    """Two selections of one row: the same scores (within 1e-6) for the indices both hold,
+    and indices held by one only must score exactly the k-th score of both (a tie at the
+    boundary, where the header leaves the choice open)."""
+    va, vb = idx_a >= 0, idx_b >= 0
+    assert va.sum() == vb.sum(), f"{what}: valid counts differ"
+    a = dict(zip(idx_a[va].tolist(), sc_a[va].tolist()))
+    b = dict(zip(idx_b[vb].tolist(), sc_b[vb].tolist()))
+    for i in a.keys() & b.keys():
+        assert abs(a[i] - b[i]) <= 1e-6 * abs(a[i]), f"{what}: index {i} scores {a[i]} vs {b[i]}"
+    only = a.keys() ^ b.keys()
+    if only:
+        kth_a, kth_b = min(a.values()), min(b.values())
+        for i in only:
+            s = a[i] if i in a else b[i]
+            assert s == kth_a == kth_b, f"{what}: index {i} selected by one call only and not tied at the k-th score"
+
+
 def test_decode_row_equals_prefill_row():
+    # the invariant of the pages' two modes: a decode step's query at position p selects what
+    # the prefill's row p selects (each call is also checked against the oracle)
     wl = W.scaled(W.prefill(), seq_lens=(3000,), q_lens=(3000,), outlier_frac=0.0)
     up = Uploaded(wl)
     pidx, psc = _run(up)
@@ -210,13 +198,13 @@ def test_decode_row_equals_prefill_row():
     q_dec = up.q[last].contiguous()
     w_dec = up.w[last].contiguous()
     didx, dsc = api.dsa_indexer_decode(q_dec, up.cache, w_dec, (3000,), (2,), wl.top_k, k_base=up.k_base)
+    api.dsa_check_device_errors()
     didx, dsc = didx.cpu().numpy(), dsc.cpu().numpy()
+    orows = up.oracle_rows([2998, 2999])
     for j, r in enumerate((2998, 2999)):
-        a = np.sort(pidx[r][pidx[r] >= 0])
-        b = np.sort(didx[j][didx[j] >= 0])
-        assert np.array_equal(a, b)
-        order_a, order_b = np.argsort(pidx[r]), np.argsort(didx[j])
-        np.testing.assert_allclose(psc[r][order_a], dsc[j][order_b], rtol=1e-6, atol=0)
+        check_row(pidx[r], psc[r], orows[j], wl.top_k, RTOL["bf16"], what=f"prefill row {r}")
+        check_row(didx[j], dsc[j], orows[j], wl.top_k, RTOL["bf16"], what=f"decode row {r}")
+        _same_set_up_to_exact_ties(pidx[r], psc[r], didx[j], dsc[j], f"row {r}")
 
 
 # ----------------------------------------------------------------------------- edge cases
@@ -263,7 +251,7 @@ def test_short_sequence_bypass_writes_the_history_and_scores_nothing(decode):
 
 
 @pytest.mark.parametrize("decode", [False, True])
-def test_caller_workspace_gives_the_same_selection_and_refuses_a_short_one(decode):
+def test_caller_workspace_matches_the_oracle_and_refuses_a_short_one(decode):
     L, q_lens = (3000, 2049, 700), ((2, 1, 1) if decode else (3000, 2049, 700))
     wl = W.scaled(W.decode() if decode else W.prefill(), seq_lens=L, q_lens=q_lens, top_k=512, seed=95)
     up = Uploaded(wl)
@@ -281,9 +269,11 @@ def test_caller_workspace_gives_the_same_selection_and_refuses_a_short_one(decod
                 idx, sc = api.dsa_indexer_prefill(up.q, up.cache, up.w, L, wl.top_k, q_scale=up.q_scale, q_lens=q_lens,
                                                   k_base=up.k_base, stream=s)
             api.dsa_check_device_errors(s)
-            for (gi, gs), (ri, rs) in zip(_sorted_rows(idx.cpu().numpy(), sc.cpu().numpy()), _sorted_rows(ref_i, ref_s)):
-                assert np.array_equal(gi, ri)
-                np.testing.assert_array_equal(gs, rs)
+            # both calls against the oracle (which keys are kept among exact ties at the k-th
+            # score is unspecified, so the two calls are not compared with each other)
+            rows = list(range(wl.total_q))
+            _check(up, ref_i, ref_s, rows)
+            _check(up, idx.cpu().numpy(), sc.cpu().numpy(), rows)
             api.dsa_set_workspace(ws[: 1 << 12], stream=s)       # far too small
             with pytest.raises(RuntimeError, match="ALLOC"):
                 api.dsa_indexer_decode(up.q, up.cache, up.w, L, q_lens, wl.top_k, q_scale=up.q_scale,
@@ -380,64 +370,16 @@ def test_edge_invalid_arguments_raise():
         api.dsa_indexer_prefill(q32, up.cache, w32, (300,), 16, q_lens=(1,))
 
 
-# ----------------------------------------------------------------------------- full-size workloads (sampled rows)
-
-def test_full_decode_batch_all_rows():
-    wl = W.decode()
-    up = Uploaded(wl)
-    idx, sc = _run(up, decode=True)
-    _check(up, idx, sc, list(range(wl.total_q)))
-
-
-def test_full_prefill_bf16_sampled_rows():
-    wl = W.prefill()
-    up = Uploaded(wl)
-    idx, sc = _run(up)
-    _check(up, idx, sc, _sample_rows(wl, n_mid=10))
-
-
-def test_full_prefill_fp8_sampled_rows():
-    wl = W.prefill8()
-    up = Uploaded(wl)
-    # the library's FP8 codes for the sampled query rows equal the oracle codec's
-    rows = _sample_rows(wl, n_mid=8)
-    bits = up.inp["q_bits"][rows].reshape(len(rows), -1)
-    codes, scale = oracle.quantize_rows(oracle.bf16_bits_to_f64(bits).astype(np.float32))
-    assert np.array_equal(up.q[rows].reshape(len(rows), -1).cpu().numpy(), codes)
-    assert np.array_equal(up.q_scale[rows].cpu().numpy(), scale)
-    idx, sc = _run(up)
-    _check(up, idx, sc, rows)
-
-
-def test_full_ragged_decode_fp8_sampled_sequences():
-    wl = W.decode8()
-    up = Uploaded(wl)
-    idx, sc = _run(up, decode=True)
-    order = np.argsort(wl.seq_lens)
-    seqs = [int(order[0]), int(order[-1]), int(order[len(order) // 2])]
-    rows = sorted(2 * b + j for b in seqs for j in (0, 1))
-    _check(up, idx, sc, rows)
-
-
 # ----------------------------------------------------------------------------- one-call host step
 
-def _sorted_rows(idx, sc):
-    out = []
-    for r in range(idx.shape[0]):
-        o = np.lexsort((idx[r], -sc[r]))
-        out.append((idx[r][o], sc[r][o]))
-    return out
-
-
 @pytest.mark.parametrize("name", ["bf16", "fp8"])
-def test_decode_host_step_equals_device_calls_two_calls_in_a_row(name):
+def test_decode_host_step_matches_the_oracle_two_calls_in_a_row(name):
     base = W.decode() if name == "bf16" else W.decode8()
     lens = [(6000, 2100, 300, 4097), (5000, 2049, 3333, 1)]
     for call, L in enumerate(lens):
         q_lens = (1, 2, 1, 1)
         wl = W.scaled(base, seq_lens=L, q_lens=q_lens, seed=50 + call)
         up = Uploaded(wl)
-        ref_i, ref_s = _run(up, decode=True)
         # the step re-appends each sequence's newest q_len keys (same values: the cache is unchanged)
         rows = np.concatenate([up.k_base[b] + np.arange(Lb - n, Lb) for b, (Lb, n) in enumerate(zip(L, q_lens))])
         k_bits = np.concatenate(up.inp["k_bits"])[rows]
@@ -451,9 +393,7 @@ def test_decode_host_step_equals_device_calls_two_calls_in_a_row(name):
         api.dsa_indexer_decode_host(q_h, w_h, k_h, rows_h, up.cache, L, q_lens, wl.top_k, oi_h, os_h,
                                     k_base=up.k_base, stream=s)
         api.dsa_check_device_errors(s)                       # synchronises the stream
-        for (gi, gs), (ri, rs) in zip(_sorted_rows(oi_h.numpy(), os_h.numpy()), _sorted_rows(ref_i, ref_s)):
-            assert np.array_equal(gi, ri)
-            np.testing.assert_array_equal(gs, rs)
+        _check(up, oi_h.numpy(), os_h.numpy(), range(wl.total_q))
 
 
 @pytest.mark.parametrize("name", ["bf16", "fp8"])
@@ -481,27 +421,14 @@ def test_decode_host_step_async_three_calls_in_flight(name):
         ev = torch.cuda.Event()
         api.dsa_indexer_decode_host(q_h, w_h, k_h, rows_h, up.cache, L, q_lens, wl.top_k, oi_h, os_h,
                                     k_base=up.k_base, stream=s, done_event=ev)
-        steps.append((q_h, w_h, oi_h, os_h, ev))
-    for q_h, w_h, oi_h, os_h, ev in steps:
+        steps.append((q_bits, w, oi_h, os_h, ev))
+    for q_bits, w, oi_h, os_h, ev in steps:
         ev.synchronize()
-        q_dev, q_scale = _device_q(up, q_h)
-        ref_i, ref_s = api.dsa_indexer_decode(q_dev, up.cache, w_h.cuda(), L, q_lens, wl.top_k, k_base=up.k_base,
-                                              q_scale=q_scale)
-        ref_i, ref_s = ref_i.cpu().numpy(), ref_s.cpu().numpy()
-        for (gi, gs), (ri, rs) in zip(_sorted_rows(oi_h.numpy(), os_h.numpy()), _sorted_rows(ref_i, ref_s)):
-            assert np.array_equal(gi, ri)
-            np.testing.assert_array_equal(gs, rs)
+        # the oracle on this step's inputs (an FP8 cache: the queries through the oracle's codec,
+        # which the host step's device quantisation matches bit for bit)
+        ref = OracleInputs(wl, dict(up.inp, q_bits=q_bits, w=w))
+        _check(ref, oi_h.numpy(), os_h.numpy(), range(wl.total_q))
     api.dsa_check_device_errors(s)
-
-
-def _device_q(up, q_h):
-    """The queries the device call takes for this cache: (bf16, None), or (E4M3 codes, scales)
-    quantised on the device as the host step does for an FP8 cache."""
-    q = q_h.cuda()
-    if not up.cache.fp8:
-        return q, None
-    codes, scale = api.dsa_quantize_rows_fp8(q.reshape(q.shape[0], -1))
-    return codes.reshape(q.shape), scale
 
 
 def test_decode_host_step_rejects_bad_arguments():
@@ -521,7 +448,7 @@ def test_decode_host_step_rejects_bad_arguments():
 
 # ----------------------------------------------------------------------------- CUDA graphs
 
-def test_graph_capture_replay_equals_eager_and_unplanned_capture_is_refused():
+def test_graph_capture_replay_matches_the_oracle_and_unplanned_capture_is_refused():
     wl = W.scaled(W.decode(), seq_lens=(3000, 2500, 40), q_lens=(1, 1, 1), seed=31)
     up = Uploaded(wl)
     s = torch.cuda.Stream()
@@ -544,10 +471,11 @@ def test_graph_capture_replay_equals_eager_and_unplanned_capture_is_refused():
     for _ in range(3):
         g.replay()
     s.synchronize()
-    # the order inside a row is unspecified: compare each row's (index, score) pairs sorted by index
-    for a_i, a_s, b_i, b_s in zip(out_i.cpu().numpy(), out_s.cpu().numpy(), eager_i.cpu().numpy(),
-                                  eager_s.cpu().numpy()):
-        oa, ob = np.argsort(a_i), np.argsort(b_i)
-        assert np.array_equal(a_i[oa], b_i[ob]) and np.array_equal(a_s[oa], b_s[ob])
+    rows = range(wl.total_q)
+    _check(up, eager_i.cpu().numpy(), eager_s.cpu().numpy(), rows)
+    _check(up, out_i.cpu().numpy(), out_s.cpu().numpy(), rows)
+    for r in rows:
+        _same_set_up_to_exact_ties(out_i[r].cpu().numpy(), out_s[r].cpu().numpy(), eager_i[r].cpu().numpy(),
+                                   eager_s[r].cpu().numpy(), f"replay row {r}")
     del g
     api.dsa_check_device_errors(s)

@@ -1,10 +1,11 @@
 """dsa_indexer_decode_noalloc: the decode entry point for callers that may not allocate
 device memory (its scratch lives in a static array inside the library).
 
-Checked through the C ABI against the regular dsa_indexer_decode on the same inputs,
-two calls in a row with different batches (the second call must not be disturbed by
-what the first left in the shared array), and for its size limit.  This file is
-collected last so that a run stopping at the first failure has run every other test.
+Checked through the C ABI against the regular dsa_indexer_decode on the same inputs and
+against the fp64 oracle, two calls in a row with different batches (the second call must
+not be disturbed by what the first left in the shared array), and for its size limit.
+This file is collected last so that a run stopping at the first failure has run every
+other test.
 """
 
 from __future__ import annotations
@@ -16,7 +17,7 @@ import torch
 from sparse_attention_token_02_b200 import api
 from sparse_attention_token_02_b200 import workloads as W
 
-from ._parity import RTOL, Uploaded
+from ._parity import RTOL, Uploaded, check_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +60,7 @@ def test_noalloc_decode_matches_regular_decode_two_calls_in_a_row():
         assert fault.cpu().tolist() == [0, 0]
         _same_selection(ref_i.cpu().numpy(), ref_s.cpu().numpy(), got_i.cpu().numpy(), got_s.cpu().numpy(),
                         wl.top_k, RTOL[wl.dtype])
+        check_rows(up, got_i.cpu().numpy(), got_s.cpu().numpy(), range(wl.total_q))
     api.dsa_check_device_errors()
 
 
@@ -73,6 +75,23 @@ def test_noalloc_decode_fp8_and_without_fault_pointer():
         torch.cuda.synchronize()
         _same_selection(ref_i.cpu().numpy(), ref_s.cpu().numpy(), got_i.cpu().numpy(), got_s.cpu().numpy(),
                         wl.top_k, RTOL[wl.dtype])
+        check_rows(up, got_i.cpu().numpy(), got_s.cpu().numpy(), range(wl.total_q))
+
+
+def test_noalloc_decode_tables_larger_than_one_parameter_chunk():
+    # 300 sequences x 2 queries: the scheduling tables (about 25 KB) reach the static array
+    # in two kernel-parameter chunks
+    rng = np.random.default_rng(7)
+    lens = tuple(int(x) for x in rng.integers(2100, 3000, 300))
+    wl = W.scaled(W.decode(), seq_lens=lens, q_lens=(2,) * len(lens), seed=23)
+    up = Uploaded(wl)
+    got_i, got_s = api.dsa_indexer_decode_noalloc(up.q, up.cache, up.w, wl.seq_lens, wl.q_lens, wl.top_k,
+                                                  q_scale=up.q_scale, k_base=up.k_base)
+    torch.cuda.synchronize()
+    got_i, got_s = got_i.cpu().numpy(), got_s.cpu().numpy()
+    rows = list(range(0, wl.total_q, 7)) + [wl.total_q - 1]
+    check_rows(up, got_i, got_s, rows)
+    api.dsa_check_device_errors()
 
 
 def test_noalloc_decode_rejects_batches_beyond_its_scratch():
