@@ -81,7 +81,11 @@ struct Cfg {
   static constexpr bool ONE_QUERY_PER_WARP = (NG == 1) && (TPA == SPLIT) && (H == 64) && !CHUNKED;
   // epilogue warps sleep inside their accumulator waits only when there are so many of
   // them that spinning would take issue slots from the ones computing
+#ifdef DSA_EPI_SLEEP_MIN
+  static constexpr bool EPI_SLEEP = NE >= DSA_EPI_SLEEP_MIN;
+#else
   static constexpr bool EPI_SLEEP = NE >= 16;
+#endif
   // the producer and MMA lanes sleep in their waits when the epilogue, not their
   // latency, sets the pace (prefill): then they leave the issue slots to the epilogue
   static constexpr bool PIPE_SLEEP = NG > 1;
@@ -90,6 +94,13 @@ struct Cfg {
   // loop leaves the epilogue slack; FP8 decode (twice the keys per byte) leaves it none, so its
   // rows are binned by a separate pass over the score rows, and prefill configurations not at all
   static constexpr bool HIST = NG == 1 && !FP8;
+  // Prefill configurations (several query groups share each K tile, 64 heads) drain their
+  // accumulators in a dedicated loop: every epilogue warp owns the same QPW query slots of
+  // every group for a whole work item, so row pointers, weight addresses and causal limits are
+  // set once per item, and the tiles whose keys precede every query of the item (all but the
+  // last one or two) run without any mask or per-query test.
+  static constexpr bool PREFILL_FAST = NG > 1 && H == 64 && EG == 1 && (TPA % SPLIT) == 0;
+  static constexpr int QPW = PREFILL_FAST ? TPA / SPLIT : 1;   // queries per warp per group
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + STAGES * K_TILE_BYTES;
@@ -203,6 +214,190 @@ __device__ unsigned long long g_pipe_stats[12];
 #else
 #define DSA_TIMED(slot, expr) (expr)
 #endif
+
+// Tuning knobs of the prefill epilogue (build-time; the defaults are the measured best):
+// accumulator chains per query in the weighted head sum, and whether a warp with several
+// query slots loads all of them before computing.
+#ifndef DSA_EPI_CHAINS
+#define DSA_EPI_CHAINS 2
+#endif
+#ifndef DSA_EPI_PAIR
+#define DSA_EPI_PAIR 0
+#endif
+
+// The same with four accumulator chains: shorter dependent FFMA2 sequences.
+__device__ __forceinline__ void relu_wsum32_c4(const uint32_t (&r)[32], const float* __restrict__ w, float2 (&a)[4]) {
+#pragma unroll
+  for (int h = 0; h < 32; h += 8) {
+    const float4 w0 = *reinterpret_cast<const float4*>(w + h);
+    const float4 w1 = *reinterpret_cast<const float4*>(w + h + 4);
+    const float2 x0 = make_float2(fmaxf(__uint_as_float(r[h]), 0.f), fmaxf(__uint_as_float(r[h + 1]), 0.f));
+    const float2 x1 = make_float2(fmaxf(__uint_as_float(r[h + 2]), 0.f), fmaxf(__uint_as_float(r[h + 3]), 0.f));
+    const float2 x2 = make_float2(fmaxf(__uint_as_float(r[h + 4]), 0.f), fmaxf(__uint_as_float(r[h + 5]), 0.f));
+    const float2 x3 = make_float2(fmaxf(__uint_as_float(r[h + 6]), 0.f), fmaxf(__uint_as_float(r[h + 7]), 0.f));
+    a[0] = __ffma2_rn(make_float2(w0.x, w0.y), x0, a[0]);
+    a[1] = __ffma2_rn(make_float2(w0.z, w0.w), x1, a[1]);
+    a[2] = __ffma2_rn(make_float2(w1.x, w1.y), x2, a[2]);
+    a[3] = __ffma2_rn(make_float2(w1.z, w1.w), x3, a[3]);
+  }
+}
+
+__device__ __forceinline__ float chains_sum(const float2 (&a)[4]) {
+  const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+  return s.x + s.y;
+}
+
+// sum_h w[h] * max(x[h], 0) over one query's 64 accumulator columns (two 32-column halves
+// already loaded), w' read from shared memory.
+__device__ __forceinline__ float relu_wsum64(const uint32_t (&r0)[32], const uint32_t (&r1)[32],
+                                            const float* __restrict__ w) {
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+  relu_wsum32(r0, w, a0, a1);
+  relu_wsum32(r1, w + 32, a0, a1);
+  return (a0.x + a0.y) + (a1.x + a1.y);
+}
+
+// The prefill epilogue for one work item over a plain cache (see Cfg::PREFILL_FAST): the
+// warp's query slots j = g * TPA + part + u * SPLIT of every group g, tiles [kt_begin, kt_end).
+// Tiles before kt_full hold only keys at or before the item's first query, so every query
+// stores every key of them; the remaining (at most two) tiles mask per query and key.
+template <class C>
+__device__ __forceinline__ void prefill_item(const LogitsArgs& args, const LogitsItem& wi, uint32_t tmem_base, int sub,
+                                             int lane, int part, const float* wq, const int64_t* rowoff,
+                                             uint64_t* acc_full, uint64_t* acc_empty, volatile int* abort_flag,
+                                             float (&ks_ring)[kScalePrefetch], uint32_t& acc_iter, bool& ok,
+                                             long long* st_) {
+  (void)st_;
+  constexpr int QPW = C::QPW, SPLIT = C::SPLIT, PF = kScalePrefetch;
+  const int groups = (wi.n_tok + C::TPA - 1) / C::TPA;
+  float* rowp[C::NG][QPW];        // score row of each slot, advanced to this thread's key of tile 0
+  const float* wp[C::NG][QPW];    // its w' in this warp's copy
+  int lastk[C::NG][QPW];          // its position: the last key it sees
+  bool live[C::NG][QPW];
+#pragma unroll
+  for (int g = 0; g < C::NG; ++g) {
+#pragma unroll
+    for (int u = 0; u < QPW; ++u) {
+      const int j = g * C::TPA + part + u * SPLIT;
+      live[g][u] = j < wi.n_tok;
+      const int jj = live[g][u] ? j : 0;
+      rowp[g][u] = args.scores + rowoff[jj] + sub * 32 + lane;
+      wp[g][u] = wq + jj * C::H;
+      lastk[g][u] = wi.pos0 + j;
+    }
+  }
+  const int pos_last = wi.pos0 + wi.n_tok - 1;
+  auto load_scale = [&](int kt) -> float {
+    const int key = kt * C::BM + sub * 32 + lane;
+    const int64_t krow = wi.k_row0 + key;
+    return (kt < wi.kt_end && key <= pos_last && krow < args.k_capacity) ? __ldg(args.k_scale + krow) : 0.f;
+  };
+  const int kt_full = max(wi.kt_begin, min(wi.kt_end, (wi.pos0 + 1) / C::BM));
+  auto tiles = [&](auto masked, int kt0, int kt1) {
+    constexpr bool kMasked = decltype(masked)::value;
+    for (int kt = kt0; kt < kt1 && ok; ++kt) {
+      const int key0 = kt * C::BM;
+      const int key = key0 + sub * 32 + lane;
+      float kscale = 1.f;
+      if constexpr (C::FP8) {
+        kscale = ks_ring[0];
+#pragma unroll
+        for (int i = 0; i + 1 < PF; ++i) ks_ring[i] = ks_ring[i + 1];
+        ks_ring[PF - 1] = load_scale(kt + PF);
+      }
+#pragma unroll
+      for (int g = 0; g < C::NG; ++g) {
+        if (g >= groups || !ok) break;
+        const int b = acc_iter % C::NBUF;
+        if (!DSA_TIMED(3, mbar_wait<C::EPI_SLEEP>(&acc_full[b], (acc_iter / C::NBUF) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        ++acc_iter;
+#ifdef DSA_PIPE_STATS
+        const long long tc0_ = clock64();
+#endif
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::ACC_COLS;
+        if constexpr (C::CHUNKED) {
+          // many epilogue warps, few registers each: one 32-column half at a time
+#pragma unroll
+          for (int u = 0; u < QPW; ++u) {
+            if (live[g][u] && (!kMasked || key0 <= lastk[g][u])) {
+              const uint32_t col = tbase + (part + u * SPLIT) * C::H;
+              uint32_t r[32];
+#if DSA_EPI_CHAINS == 4
+              float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
+              tmem_ld_32x32b_x32(col, r);
+              tmem_ld_wait();
+              relu_wsum32_c4(r, wp[g][u], a);
+              tmem_ld_32x32b_x32(col + 32, r);
+              tmem_ld_wait();
+              relu_wsum32_c4(r, wp[g][u] + 32, a);
+              const float v = chains_sum(a) * kscale;
+#else
+              float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+              tmem_ld_32x32b_x32(col, r);
+              tmem_ld_wait();
+              relu_wsum32(r, wp[g][u], a0, a1);
+              tmem_ld_32x32b_x32(col + 32, r);
+              tmem_ld_wait();
+              relu_wsum32(r, wp[g][u] + 32, a0, a1);
+              const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+#endif
+              if (!kMasked || key <= lastk[g][u]) rowp[g][u][key0] = v;
+            }
+          }
+        } else if (DSA_EPI_PAIR && QPW == 2) {
+          // both slots' 128 columns in flight behind one wait, then two independent sums
+          uint32_t r[2][2][32];
+          bool go[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            go[u] = live[g][u] && (!kMasked || key0 <= lastk[g][u]);
+            const uint32_t col = tbase + (part + u * SPLIT) * C::H;
+            if (go[u]) {
+              tmem_ld_32x32b_x32(col, r[u][0]);
+              tmem_ld_32x32b_x32(col + 32, r[u][1]);
+            }
+          }
+          if (go[0] || go[1]) tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (go[u]) {
+              const float v = relu_wsum64(r[u][0], r[u][1], wp[g][u]) * kscale;
+              if (!kMasked || key <= lastk[g][u]) rowp[g][u][key0] = v;
+            }
+          }
+        } else {
+          // one slot at a time, its 64 columns in flight behind one wait
+#pragma unroll
+          for (int u = 0; u < QPW; ++u) {
+            if (live[g][u] && (!kMasked || key0 <= lastk[g][u])) {
+              const uint32_t col = tbase + (part + u * SPLIT) * C::H;
+              uint32_t r0[32], r1[32];
+              tmem_ld_32x32b_x32(col, r0);
+              tmem_ld_32x32b_x32(col + 32, r1);
+              tmem_ld_wait();
+              const float v = relu_wsum64(r0, r1, wp[g][u]) * kscale;
+              if (!kMasked || key <= lastk[g][u]) rowp[g][u][key0] = v;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+#ifdef DSA_PIPE_STATS
+        st_[4] += clock64() - tc0_;
+#endif
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+      }
+    }
+  };
+  tiles(std::false_type{}, wi.kt_begin, kt_full);
+  tiles(std::true_type{}, kt_full, wi.kt_end);
+}
+
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
@@ -438,6 +633,18 @@ logits_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant_
 #pragma unroll
         for (int i = 0; i < PF; ++i) ks_ring[i] = load_scale(wi.kt_begin + i);
       }
+      if constexpr (C::PREFILL_FAST) {
+        if (cmp == 1) {
+#ifdef DSA_PIPE_STATS
+          prefill_item<C>(args, wi, tmem_base, sub, lane, part, wq, rowoff, acc_full, acc_empty, abort_flag,
+                          ks_ring, acc_iter, ok, st_);
+#else
+          prefill_item<C>(args, wi, tmem_base, sub, lane, part, wq, rowoff, acc_full, acc_empty, abort_flag,
+                          ks_ring, acc_iter, ok, nullptr);
+#endif
+          continue;
+        }
+      }
       // the tile loop, compiled twice: plain causal limits (one add per query) and limits
       // over a compressed cache (a division), so the plain loop carries no compression test
       auto tile_loop = [&](auto compressed) {
@@ -647,7 +854,7 @@ cudaError_t launch_cfg(const LogitsLaunch& L, const CUtensorMap& tk, const CUten
 #define DSA_PB16_EG 1
 #endif
 #ifndef DSA_PF8_NE
-#define DSA_PF8_NE 16
+#define DSA_PF8_NE 8
 #endif
 #ifndef DSA_PF8_STAGES
 #define DSA_PF8_STAGES 4

@@ -21,6 +21,7 @@
 //     DSMEM atomic per CTA gives each thread its output slots.
 // Output order inside a row is unspecified (the selection is a set).
 #include <cooperative_groups.h>
+#include <type_traits>
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -212,20 +213,29 @@ __device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, 
   __syncthreads();
   const uint32_t n_sel_up = n_up + (need - ls.need);     // keys above the final interval
   const uint32_t first_in = base + n_sel_up;             // slots of interval keys start here
+  // slots per warp: one atomic per counter and warp (every thread calls f the same number of
+  // times, so the ballots see the whole warp)
+  const uint32_t lane_lt = (1u << (threadIdx.x & 31)) - 1u;
   for_candidates<kGlobalCand, true, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t ix, bool valid) {
-    if (!valid) return;
-    if (kk > ls.hi) {
-      const uint32_t slot = base + atomicAdd(ctr_a, 1u);
+    const bool up = valid && kk > ls.hi;
+    const bool in = valid && !up && kk >= ls.lo;
+    const uint32_t bu = __ballot_sync(0xffffffffu, up), bi = __ballot_sync(0xffffffffu, in);
+    uint32_t su = 0u, si = 0u;
+    if ((threadIdx.x & 31) == 0) {
+      if (bu) su = atomicAdd(ctr_a, static_cast<uint32_t>(__popc(bu)));
+      if (bi) si = atomicAdd(ctr_b, static_cast<uint32_t>(__popc(bi)));
+    }
+    su = __shfl_sync(0xffffffffu, su, 0) + __popc(bu & lane_lt);
+    si = __shfl_sync(0xffffffffu, si, 0) + __popc(bi & lane_lt);
+    if (up) {
+      const uint32_t slot = base + su;
       if (slot < first_in) {
         oi[slot] = ix;
         os[slot] = key_to_float(kk);
       }
-    } else if (kk >= ls.lo) {
-      const uint32_t t = atomicAdd(ctr_b, 1u);
-      if (t < ls.need) {
-        oi[first_in + t] = ix;
-        os[first_in + t] = key_to_float(kk);
-      }
+    } else if (in && si < ls.need) {
+      oi[first_in + si] = ix;
+      os[first_in + si] = key_to_float(kk);
     }
   });
   __syncthreads();
@@ -769,6 +779,20 @@ constexpr int kRowCap = 4096;                             // interval keys gathe
 constexpr int kRowShift0 = 20;                            // first level: 4096 bins of the top 12 bits
 constexpr int kRowBins0 = 1 << (32 - kRowShift0);
 constexpr size_t kRowSmemBytes = (kRowBins0 + 2 * kRowCap) * sizeof(uint32_t);
+// The row streams from HBM with only one iteration of loads in flight per thread; the L2 is
+// asked for the row kRowAhead iterations ahead (one bulk prefetch per iteration, by one
+// thread), so the loads find the row there instead of waiting on HBM.
+constexpr int kRowAhead = 3;
+
+// Bulk L2 prefetch of iteration `it` of a row of n keys (the row's storage is n rounded up to
+// 4 floats, so the prefetch never leaves it).
+__device__ __forceinline__ void row_prefetch(const float* src, int n, int it) {
+  const int first = it * kRowIter;
+  if (first >= n) return;
+  const int last = min(n, first + kRowIter);
+  const uint32_t bytes = static_cast<uint32_t>(((last - first + 3) & ~3) * sizeof(float));
+  l2_prefetch_bulk(src + first, bytes);
+}
 static_assert(kRowBins0 % kRowThreads == 0 && kBins % kRowThreads == 0, "bins per thread");
 
 __device__ __forceinline__ void row_load(const float* src, int n, int base, float4 (&f)[kRowEPT / 4]) {
@@ -791,10 +815,19 @@ __device__ bool row_sampled_select(const float* src, int n, uint32_t k, int32_t*
   const int block = 64 * ((n + 65535) / 65536);
   const int n_blocks = (n + block - 1) / block;
   uint32_t smin = 0xFFFFFFFFu, smax = 0u, s_local = 0u;
-  for (int b = tid; b < n_blocks; b += kRowThreads) {
+  constexpr int kSampleLoads = kRowCap / 4 / kRowThreads;   // n_blocks <= kRowCap / 4
+  float4 sf[kSampleLoads];
+#pragma unroll
+  for (int j = 0; j < kSampleLoads; ++j) {                  // every load in flight before any is used
+    const int b = tid + j * kRowThreads;
+    sf[j] = b < n_blocks ? __ldcs(reinterpret_cast<const float4*>(src + b * block)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int j = 0; j < kSampleLoads; ++j) {
+    const int b = tid + j * kRowThreads;
+    if (b >= n_blocks) break;
     const int i = b * block;
-    const float4 f = __ldcs(reinterpret_cast<const float4*>(src + i));
-    const float fv[4] = {f.x, f.y, f.z, f.w};
+    const float fv[4] = {sf[j].x, sf[j].y, sf[j].z, sf[j].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const bool valid = i + e < n;
@@ -848,34 +881,25 @@ __device__ bool row_sampled_select(const float* src, int n, uint32_t k, int32_t*
   if (*lvl_bin == kNotFound) return false;    // the sample holds fewer than r keys
   const uint32_t tau = lo_s + (*lvl_bin << shift);
   const float tau_f = key_to_float(tau);
-  if (tid == 0) {
-    *ctr_a = 0u;                              // gathered keys
-    *ctr_b = 0u;                              // largest gathered key
-    *ctr_c = 0xFFFFFFFFu;                     // smallest gathered key
-  }
+  if (tid == 0) *ctr_a = 0u;                  // gathered keys
   __syncthreads();
 
-  // ---- one pass: every key >= tau into shared memory (slots: warp scan + one atomic per warp).
-  // {f >= tau_f} is closed upwards in key order (key order refines float order), so it holds
-  // the k largest keys as soon as it has k elements.
-  uint32_t my_max = 0u, my_min = 0xFFFFFFFFu;
+  // ---- one pass: every key >= tau into shared memory (slots: warp scan + one atomic per
+  // warp).  {f >= tau_f} is closed upwards in key order (key order refines float order), so it
+  // holds the k largest keys as soon as it has k elements.
   float4 cur[kRowEPT / 4];
   row_load(src, n, 0, cur);
-  for (int base = 0; base < n; base += kRowIter) {
-    float4 nxt[kRowEPT / 4];
-    if (base + kRowIter < n) {
-      row_load(src, n, base + kRowIter, nxt);
-    } else {
-#pragma unroll
-      for (int v = 0; v < kRowEPT / 4; ++v) nxt[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+  auto gather = [&](auto tail, int base) {
+    constexpr bool kTail = decltype(tail)::value;   // the last iteration: positions past n exist
     uint32_t sel = 0u;
 #pragma unroll
     for (int v = 0; v < kRowEPT / 4; ++v) {
       const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        sel |= static_cast<uint32_t>(fv[e] >= tau_f && base + (v * kRowThreads + tid) * 4 + e < n) << (v * 4 + e);
+      for (int e = 0; e < 4; ++e) {
+        const bool hit = fv[e] >= tau_f && (!kTail || base + (v * kRowThreads + tid) * 4 + e < n);
+        sel |= static_cast<uint32_t>(hit) << (v * 4 + e);
+      }
     }
     const uint32_t mine = __popc(sel);
     uint32_t incl = mine;
@@ -887,41 +911,63 @@ __device__ bool row_sampled_select(const float* src, int n, uint32_t k, int32_t*
     uint32_t wbase = 0u;
     if (lane == 31 && incl) wbase = atomicAdd(ctr_a, incl);
     uint32_t slot = __shfl_sync(0xffffffffu, wbase, 31) + incl - mine;
-    if (sel) {
+    // the selected keys, float4 by float4: a float4 with no selected key costs one test
 #pragma unroll
-      for (int v = 0; v < kRowEPT / 4; ++v) {
+    for (int v = 0; v < kRowEPT / 4; ++v) {
+      const uint32_t nib = (sel >> (4 * v)) & 0xFu;
+      if (nib) {
         const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
+        const int pos0 = base + (v * kRowThreads + tid) * 4;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          if ((sel >> (v * 4 + e)) & 1u) {
-            const uint32_t kk = float_to_key(fv[e]);
-            my_max = max(my_max, kk);
-            my_min = min(my_min, kk);
+          if ((nib >> e) & 1u) {
             if (slot < static_cast<uint32_t>(kRowCap)) {
-              cand_key[slot] = kk;
-              cand_idx[slot] = base + (v * kRowThreads + tid) * 4 + e;
+              cand_key[slot] = float_to_key(fv[e]);
+              cand_idx[slot] = pos0 + e;
             }
             ++slot;
           }
         }
       }
     }
+  };
+  int base = 0;
+  for (; base + kRowIter < n; base += kRowIter) {        // every position of this iteration is < n
+    if (tid == 0) row_prefetch(src, n, base / kRowIter + kRowAhead);
+    float4 nxt[kRowEPT / 4];
+    row_load(src, n, base + kRowIter, nxt);
+    gather(std::false_type{}, base);
 #pragma unroll
     for (int v = 0; v < kRowEPT / 4; ++v) cur[v] = nxt[v];
+  }
+  gather(std::true_type{}, base);
+  __syncthreads();
+  const uint32_t c = *ctr_a;
+  if (c < k || c > static_cast<uint32_t>(kRowCap)) return false;   // tau missed: exact passes instead
+  // the gathered keys' range
+  uint32_t my_max = 0u, my_min = 0xFFFFFFFFu;
+  for (uint32_t i = tid; i < c; i += kRowThreads) {
+    const uint32_t kk = cand_key[i];
+    my_max = max(my_max, kk);
+    my_min = min(my_min, kk);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
     my_min = min(my_min, __shfl_xor_sync(0xffffffffu, my_min, o));
   }
-  if (lane == 0 && my_max) {
+  if (tid == 0) {
+    *ctr_b = 0u;                              // largest gathered key
+    *ctr_c = 0xFFFFFFFFu;                     // smallest gathered key
+  }
+  __syncthreads();
+  if (lane == 0) {
     atomicMax(ctr_b, my_max);
     atomicMin(ctr_c, my_min);
   }
   __syncthreads();
-  const uint32_t c = *ctr_a, kmax = *ctr_b, kmin = *ctr_c;
+  const uint32_t kmax = *ctr_b, kmin = *ctr_c;
   __syncthreads();                            // every thread has read the counters
-  if (c < k || c > static_cast<uint32_t>(kRowCap)) return false;   // tau missed: exact passes instead
   const bool ok = rank0_select<false, kRowThreads>(cand_key, cand_idx, c, 0u, kmin, kmax, k, 0u, oi, os, hist,
                                                    warp_sums, lvl_bin, lvl_above, lvl_cnt, ctr_a, ctr_b);
   if (!ok && tid == 0) record_error(err, DSA_DEVERR_TOPK, row);
@@ -949,6 +995,8 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
   uint32_t cnt = static_cast<uint32_t>(n);                // keys inside [lo, hi]
   int shift = kRowShift0;
   grid_dependency_wait();                                 // the scores come from the previous kernel
+  if (tid == 0)
+    for (int it = 0; it < kRowAhead; ++it) row_prefetch(src, n, it);
   if (n > kRowCap && k <= static_cast<uint32_t>(kRowCap) / 2 &&
       row_sampled_select(src, n, k, oi, os, hist, cand_key, cand_idx, warp_sums, &lvl_bin, &lvl_above, &lvl_cnt,
                          &ctr_a, &ctr_b, &ctr_c, a.err, row))
@@ -968,6 +1016,7 @@ __global__ void __launch_bounds__(kRowThreads, 4) topk_row_kernel(const TopkArgs
     float4 cur[kRowEPT / 4];
     row_load(src, n, 0, cur);
     for (int base = 0; base < n; base += kRowIter) {
+      if (tid == 0) row_prefetch(src, n, base / kRowIter + kRowAhead);
       float4 nxt[kRowEPT / 4];
       if (base + kRowIter < n) {
         row_load(src, n, base + kRowIter, nxt);

@@ -107,6 +107,13 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Bulk prefetch of global memory [ptr, ptr + bytes) into the L2; nothing to wait for.  ptr and
+// bytes must be multiples of 16.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(ptr)), "r"(bytes)
+               : "memory");
+}
+
 // 2-D tiled bulk tensor load into this CTA's shared memory, completing on `bar`.
 // x is the innermost (contiguous) coordinate in elements; callers keep
 // x * element_size a multiple of 16 bytes.
