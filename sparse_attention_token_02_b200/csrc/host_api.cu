@@ -636,7 +636,8 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     tpa = 4;
     ng = 2;
   }
-  if (!logits_config_supported(H, D, fp8, tpa, ng))
+  const bool prefill_items = !decode_sched && H != 4;
+  if (!logits_config_supported(H, D, fp8, tpa, ng, prefill_items))
     return fail(DSA_ERR_UNSUPPORTED, "no %s kernel for H_I=%d, d_I=%d, dtype=%s", decode_sched ? "decode" : "prefill",
                 H, D, fp8 ? "fp8" : "bf16");
 
@@ -739,7 +740,7 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
   la.row_hist = d_hist;
   la.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   la.err = c->d_err;
-  LogitsLaunch L{H, D, fp8, tpa, ng, static_cast<int>(p.cta_items.size()) - 1, stream};
+  LogitsLaunch L{H, D, fp8, tpa, ng, static_cast<int>(p.cta_items.size()) - 1, stream, prefill_items};
   // inside a capture the events must become event-record nodes of the graph
   const unsigned ev_flags = capturing ? cudaEventRecordExternal : cudaEventRecordDefault;
   if (g_prof[0]) DSA_CUDA_TRY(cudaEventRecordWithFlags(g_prof[0], stream, ev_flags), "cudaEventRecord");
@@ -1332,7 +1333,7 @@ extern "C" dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const d
   const bool fp8 = kc->dtype == DSA_FP8_E4M3;
   const int H = q->H_I, D = kc->d_I;
   const int tpa = logits_queries_per_item(H, D, false, v.max_q_len);
-  if (!logits_config_supported(H, D, fp8, tpa, 1))
+  if (!logits_config_supported(H, D, fp8, tpa, 1, false))
     return fail(DSA_ERR_UNSUPPORTED, "no decode kernel for H_I=%d, d_I=%d, dtype=%s", H, D, fp8 ? "fp8" : "bf16");
 
   int dev = 0;
@@ -1375,7 +1376,7 @@ extern "C" dsa_status_t dsa_indexer_decode_noalloc(const dsa_query_t* q, const d
   la.scores = d_scores;
   la.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   la.err = err;
-  LogitsLaunch L{H, D, fp8, tpa, 1, static_cast<int>(p.cta_items.size()) - 1, stream};
+  LogitsLaunch L{H, D, fp8, tpa, 1, static_cast<int>(p.cta_items.size()) - 1, stream, false};
   DSA_CUDA_TRY(launch_logits(L, tk, tq, la), "logits kernel launch");
   g_launches += L.grid > 0;
   TopkArgs ta{};

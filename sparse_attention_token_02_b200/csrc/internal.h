@@ -98,11 +98,13 @@ struct LogitsLaunch {
   int ng;      // accumulators (query groups) per work item
   int grid;
   cudaStream_t stream;
+  bool prefill;   // prefill work items (a query block over its causal range), else decode
 };
+
 
 cudaError_t launch_logits(const LogitsLaunch& L, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q,
                           const LogitsArgs& a);
-bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng);
+bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng, bool prefill);
 
 // Top-k over rows longer than top_k: one cluster of `cluster` CTAs per row,
 // `ept` keys per thread held in registers.

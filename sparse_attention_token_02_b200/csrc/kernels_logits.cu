@@ -39,8 +39,9 @@ constexpr int kScalePrefetch = 4;   // tiles of FP8 key scales in flight ahead o
 #define DSA_TMEM_X64 0                  // one 64-column TMEM load per query instead of two
 #endif
 
-template <int H_, int D_, bool FP8_, int TPA_, int NG_, int NE_, int STAGES_, int EG_ = 1>
+template <int H_, int D_, bool FP8_, int TPA_, int NG_, int NE_, int STAGES_, int EG_ = 1, bool PF_ = false>
 struct Cfg {
+  static constexpr bool PF = PF_;                   // a prefill configuration (else decode)
   static constexpr int H = H_, D = D_, TPA = TPA_, NG = NG_, NE = NE_, STAGES = STAGES_;
   // Epilogue warps form EG groups; group g drains accumulators g, g+EG, ... so EG
   // accumulators are drained at once.  Inside a group, the SPLIT warps that share a TMEM
@@ -78,7 +79,7 @@ struct Cfg {
   static constexpr bool CHUNKED = THREADS > 384;
   // every epilogue warp owns exactly one query of the work item: its head weights stay
   // in registers for the whole item
-  static constexpr bool ONE_QUERY_PER_WARP = (NG == 1) && (TPA == SPLIT) && (H == 64) && !CHUNKED;
+  static constexpr bool ONE_QUERY_PER_WARP = (NG == 1) && (TPA == SPLIT) && (H == 64) && !CHUNKED && !PF;
   // epilogue warps sleep inside their accumulator waits only when there are so many of
   // them that spinning would take issue slots from the ones computing
 #ifdef DSA_EPI_SLEEP_MIN
@@ -88,18 +89,18 @@ struct Cfg {
 #endif
   // the producer and MMA lanes sleep in their waits when the epilogue, not their
   // latency, sets the pace (prefill): then they leave the issue slots to the epilogue
-  static constexpr bool PIPE_SLEEP = NG > 1;
+  static constexpr bool PIPE_SLEEP = PF;
   // decode configurations can bin every row for the top-k (prefill ones compile no such code)
   // bf16 decode configurations bin every row for the top-k in the epilogue, where the HBM-bound
   // loop leaves the epilogue slack; FP8 decode (twice the keys per byte) leaves it none, so its
   // rows are binned by a separate pass over the score rows, and prefill configurations not at all
-  static constexpr bool HIST = NG == 1 && !FP8;
+  static constexpr bool HIST = NG == 1 && !FP8 && !PF;
   // Prefill configurations (several query groups share each K tile, 64 heads) drain their
   // accumulators in a dedicated loop: every epilogue warp owns the same QPW query slots of
   // every group for a whole work item, so row pointers, weight addresses and causal limits are
   // set once per item, and the tiles whose keys precede every query of the item (all but the
   // last one or two) run without any mask or per-query test.
-  static constexpr bool PREFILL_FAST = NG > 1 && H == 64 && EG == 1 && (TPA % SPLIT) == 0;
+  static constexpr bool PREFILL_FAST = PF && H == 64 && EG == 1 && (TPA % SPLIT) == 0;
   static constexpr int QPW = PREFILL_FAST ? TPA / SPLIT : 1;   // queries per warp per group
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_K = 0;
@@ -224,6 +225,10 @@ __device__ unsigned long long g_pipe_stats[12];
 #ifndef DSA_EPI_PAIR
 #define DSA_EPI_PAIR 0
 #endif
+// 1: the next slot's (or half's) TMEM columns are loaded while the current ones are summed
+#ifndef DSA_EPI_PIPE
+#define DSA_EPI_PIPE 0
+#endif
 
 // The same with four accumulator chains: shorter dependent FFMA2 sequences.
 __device__ __forceinline__ void relu_wsum32_c4(const uint32_t (&r)[32], const float* __restrict__ w, float2 (&a)[4]) {
@@ -319,7 +324,42 @@ __device__ __forceinline__ void prefill_item(const LogitsArgs& args, const Logit
 #endif
         tc_fence_after();
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + b * C::ACC_COLS;
-        if constexpr (C::CHUNKED) {
+        if constexpr (C::CHUNKED && DSA_EPI_PIPE && QPW == 1) {
+          // one slot: its second half loads while the first is summed
+          if (live[g][0] && (!kMasked || key0 <= lastk[g][0])) {
+            const uint32_t col = tbase + part * C::H;
+            uint32_t ra[32], rb[32];
+            float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+            tmem_ld_32x32b_x32(col, ra);
+            tmem_ld_wait();
+            tmem_ld_32x32b_x32(col + 32, rb);
+            relu_wsum32(ra, wp[g][0], a0, a1);
+            tmem_ld_wait();
+            relu_wsum32(rb, wp[g][0] + 32, a0, a1);
+            const float v = ((a0.x + a0.y) + (a1.x + a1.y)) * kscale;
+            if (!kMasked || key <= lastk[g][0]) rowp[g][0][key0] = v;
+          }
+        } else if constexpr (!C::CHUNKED && DSA_EPI_PIPE && QPW == 2) {
+          // two slots: the second slot's 64 columns load while the first slot is summed (both
+          // slots' columns are read whether or not the slot holds a query: harmless, and it keeps
+          // the loads unconditional)
+          const uint32_t col0 = tbase + part * C::H, col1 = tbase + (part + SPLIT) * C::H;
+          uint32_t ra0[32], ra1[32], rb0[32], rb1[32];
+          tmem_ld_32x32b_x32(col0, ra0);
+          tmem_ld_32x32b_x32(col0 + 32, ra1);
+          tmem_ld_wait();
+          tmem_ld_32x32b_x32(col1, rb0);
+          tmem_ld_32x32b_x32(col1 + 32, rb1);
+          if (live[g][0] && (!kMasked || key0 <= lastk[g][0])) {
+            const float v = relu_wsum64(ra0, ra1, wp[g][0]) * kscale;
+            if (!kMasked || key <= lastk[g][0]) rowp[g][0][key0] = v;
+          }
+          tmem_ld_wait();
+          if (live[g][1] && (!kMasked || key0 <= lastk[g][1])) {
+            const float v = relu_wsum64(rb0, rb1, wp[g][1]) * kscale;
+            if (!kMasked || key <= lastk[g][1]) rowp[g][1][key0] = v;
+          }
+        } else if constexpr (C::CHUNKED) {
           // many epilogue warps, few registers each: one 32-column half at a time
 #pragma unroll
           for (int u = 0; u < QPW; ++u) {
@@ -878,8 +918,8 @@ cudaError_t launch_cfg(const LogitsLaunch& L, const CUtensorMap& tk, const CUten
 #define DSA_D2F8_EG 1
 #endif
 //                                  H   D   FP8   TPA NG NE               STAGES               EG
-using CfgPrefillBf16   = Cfg<64, 128, false, 4, 2, DSA_PB16_NE,  DSA_PB16_STAGES,  DSA_PB16_EG>;
-using CfgPrefillFp8    = Cfg<64, 128, true,  4, 2, DSA_PF8_NE,   DSA_PF8_STAGES,   DSA_PF8_EG>;
+using CfgPrefillBf16   = Cfg<64, 128, false, 4, 2, DSA_PB16_NE,  DSA_PB16_STAGES,  DSA_PB16_EG, true>;
+using CfgPrefillFp8    = Cfg<64, 128, true,  4, 2, DSA_PF8_NE,   DSA_PF8_STAGES,   DSA_PF8_EG, true>;
 using CfgDecode1Bf16   = Cfg<64, 128, false, 1, 1, DSA_D1B16_NE, DSA_D1B16_STAGES>;
 using CfgDecode2Bf16   = Cfg<64, 128, false, 2, 1, 8, 5>;
 using CfgDecode4Bf16   = Cfg<64, 128, false, 4, 1, 8, 4>;
@@ -907,9 +947,9 @@ extern "C" __attribute__((visibility("default"))) int dsa_debug_pipe_stats(unsig
 }
 #endif
 
-bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng) {
+bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng, bool prefill) {
   if (H == 64 && D == 128) {
-    if (ng == 2 && tpa == 4) return true;
+    if (prefill) return tpa == 4 && ng == 2;
     if (ng == 1 && (tpa == 1 || tpa == 2 || tpa == 4)) return true;
   }
   if (H == 4 && D == 64 && !fp8 && tpa == 64 && ng == 1) return true;
@@ -920,8 +960,10 @@ cudaError_t launch_logits(const LogitsLaunch& L, const CUtensorMap& tk, const CU
                           const LogitsArgs& a) {
   if (L.grid <= 0) return cudaSuccess;
   if (L.H == 64 && L.D == 128) {
-    if (L.ng == 2 && L.tpa == 4)
+    if (L.prefill) {
+      if (L.tpa != 4 || L.ng != 2) return cudaErrorInvalidValue;
       return L.fp8 ? launch_cfg<CfgPrefillFp8>(L, tk, tq, a) : launch_cfg<CfgPrefillBf16>(L, tk, tq, a);
+    }
     if (L.ng == 1) {
       switch (L.tpa) {
         case 1: return L.fp8 ? launch_cfg<CfgDecode1Fp8>(L, tk, tq, a) : launch_cfg<CfgDecode1Bf16>(L, tk, tq, a);
