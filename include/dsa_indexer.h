@@ -15,8 +15,8 @@
  * - Pointers named "device" are CUDA device pointers on the current device;
  *   "host" pointers are read synchronously during the call and may be reused
  *   as soon as it returns -- except the *_host buffers of the host-step calls
- *   (dsa_indexer_decode_host and _async), which are copied asynchronously and
- *   stay in use until the step completes.  Device pointers passed to the
+ *   (dsa_indexer_decode_host, dsa_indexer_prefill_host and their _async forms),
+ *   which are copied asynchronously and stay in use until the step completes.  Device pointers passed to the
  *   tensor-core path (the cache, the queries) must be 16-byte aligned.
  * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
  *   only enqueues work on it; outputs are valid once the stream has reached
@@ -202,6 +202,28 @@ DSA_API dsa_status_t dsa_indexer_decode_host_async(const dsa_query_t* q, const d
                                                    const int64_t* dst_rows_host, int32_t n_new,
                                                    const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
                                                    float* out_score_host, void* stream, void* done_event);
+
+/*
+ * The prefill counterparts of the two host-step calls above: the same copies, slots, copy
+ * streams and ordering, with the scoring and selection of dsa_indexer_prefill (any q_lens,
+ * q_lens may be NULL: every key of a sequence has its query).  A prefill step moves much more
+ * than a decode step (the 65 536-token FP8 prefill uploads 1 GB of bf16 queries and reads 1 GB
+ * of selection back), so the copies of one step overlap the kernels of its neighbours: the
+ * uploads of step i+1 and the read-back of step i-1 (with the _async form) run while step i
+ * scores.  Each slot holds a step's inputs and outputs on the device (both slots together about
+ * 2 x (bf16 queries + selection) bytes, grown on demand with cudaMalloc).
+ * ("Study MLA Indexer", 数学流: [L, L] logits then arg top-k [L, k], for a prompt of L tokens.)
+ */
+DSA_API dsa_status_t dsa_indexer_prefill_host(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                              const void* k_new_host, dsa_dtype_t k_new_dtype,
+                                              const int64_t* dst_rows_host, int32_t n_new, const dsa_batch_t* batch,
+                                              int32_t top_k, int32_t* out_idx_host, float* out_score_host,
+                                              void* stream);
+DSA_API dsa_status_t dsa_indexer_prefill_host_async(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                                    const void* k_new_host, dsa_dtype_t k_new_dtype,
+                                                    const int64_t* dst_rows_host, int32_t n_new,
+                                                    const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
+                                                    float* out_score_host, void* stream, void* done_event);
 
 /*
  * The scores alone, without selection (the first page's index_scores, §3):

@@ -26,6 +26,8 @@ EXPORTED = (
     "dsa_indexer_decode_noalloc",
     "dsa_indexer_decode_host",
     "dsa_indexer_decode_host_async",
+    "dsa_indexer_prefill_host",
+    "dsa_indexer_prefill_host_async",
     "dsa_indexer_decode_compressed",
     "dsa_indexer_prefill_compressed",
     "dsa_indexer_kcache_append_rope",
@@ -94,11 +96,13 @@ def load() -> ctypes.CDLL:
         fn.restype = st
     lib.dsa_indexer_decode_noalloc.argtypes = [P(Query), P(KCache), V, P(Batch), I32, V, V, V, V]
     lib.dsa_indexer_decode_noalloc.restype = st
-    lib.dsa_indexer_decode_host.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V, V]
-    lib.dsa_indexer_decode_host.restype = st
-    lib.dsa_indexer_decode_host_async.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V,
-                                                  V, V]
-    lib.dsa_indexer_decode_host_async.restype = st
+    for name in ("dsa_indexer_decode_host", "dsa_indexer_prefill_host"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V, V]
+        fn.restype = st
+        fn = getattr(lib, name + "_async")
+        fn.argtypes = [P(Query), P(KCache), V, V, ctypes.c_int, V, I32, P(Batch), I32, V, V, V, V]
+        fn.restype = st
     lib.dsa_indexer_decode_compressed.argtypes = [P(Query), P(KCache), V, P(Batch), I32, I32, V, V, V]
     lib.dsa_indexer_decode_compressed.restype = st
     lib.dsa_indexer_prefill_compressed.argtypes = [P(Query), P(KCache), V, P(Batch), I32, I32, V, V, V]

@@ -188,6 +188,32 @@ def dsa_indexer_decode_noalloc(q, cache: IndexerKCache, w, seq_lens, q_lens, top
     return out_idx, out_score
 
 
+def _host_step(fn_name, q_host, w_host, k_new_host, dst_rows_host, cache, batch, top_k, out_idx_host,
+               out_score_host, q_scale_host, stream, done_event):
+    for t in (q_host, w_host, k_new_host, dst_rows_host, out_idx_host, out_score_host, q_scale_host):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{fn_name} takes contiguous host tensors")
+    if w_host.dtype != torch.float32 or out_score_host.dtype != torch.float32 or out_idx_host.dtype != torch.int32:
+        raise TypeError("w and out_score must be fp32, out_idx int32")
+    if dst_rows_host.dtype != torch.int64:
+        raise TypeError("dst_rows must be int64")
+    if q_host.dim() != 3:
+        raise ValueError("q must be [T_total, H_I, d_I]")
+    qq = Query(q_host.data_ptr(), q_scale_host.data_ptr() if q_scale_host is not None else None, _dtype_code(q_host),
+               q_host.shape[1], q_host.shape[2])
+    kc = cache.c()
+    n_new = int(k_new_host.shape[0]) if k_new_host is not None else 0
+    args = (ctypes.byref(qq), ctypes.byref(kc), _ptr(w_host), _ptr(k_new_host),
+            _dtype_code(k_new_host) if n_new else DSA_BF16, _ptr(dst_rows_host), n_new, ctypes.byref(batch.c), top_k,
+            _ptr(out_idx_host), _ptr(out_score_host), _stream(stream))
+    if done_event is None:
+        check(getattr(_lib.load(), fn_name)(*args))
+        return
+    if not done_event.cuda_event:               # torch creates its events on their first record
+        done_event.record(torch.cuda.current_stream() if stream is None else stream)
+    check(getattr(_lib.load(), fn_name + "_async")(*args, ctypes.c_void_p(done_event.cuda_event)))
+
+
 def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: IndexerKCache, seq_lens, q_lens,
                             top_k, out_idx_host, out_score_host, q_scale_host=None, k_base=None, stream=None,
                             done_event=None):
@@ -200,29 +226,19 @@ def dsa_indexer_decode_host(q_host, w_host, k_new_host, dst_rows_host, cache: In
     or, with ``done_event`` (a torch.cuda.Event; dsa_indexer_decode_host_async), once that event
     has completed, while ``stream`` goes on without waiting for the read-back.  Pinned host
     tensors keep the copies asynchronous."""
-    for t in (q_host, w_host, k_new_host, dst_rows_host, out_idx_host, out_score_host, q_scale_host):
-        if t is not None and (t.is_cuda or not t.is_contiguous()):
-            raise ValueError("dsa_indexer_decode_host takes contiguous host tensors")
-    if w_host.dtype != torch.float32 or out_score_host.dtype != torch.float32 or out_idx_host.dtype != torch.int32:
-        raise TypeError("w and out_score must be fp32, out_idx int32")
-    if dst_rows_host.dtype != torch.int64:
-        raise TypeError("dst_rows must be int64")
-    if q_host.dim() != 3:
-        raise ValueError("q must be [T_total, H_I, d_I]")
-    b = _batch(seq_lens, q_lens, k_base)
-    qq = Query(q_host.data_ptr(), q_scale_host.data_ptr() if q_scale_host is not None else None, _dtype_code(q_host),
-               q_host.shape[1], q_host.shape[2])
-    kc = cache.c()
-    n_new = int(k_new_host.shape[0]) if k_new_host is not None else 0
-    args = (ctypes.byref(qq), ctypes.byref(kc), _ptr(w_host), _ptr(k_new_host),
-            _dtype_code(k_new_host) if n_new else DSA_BF16, _ptr(dst_rows_host), n_new, ctypes.byref(b.c), top_k,
-            _ptr(out_idx_host), _ptr(out_score_host), _stream(stream))
-    if done_event is None:
-        check(_lib.load().dsa_indexer_decode_host(*args))
-        return
-    if not done_event.cuda_event:               # torch creates its events on their first record
-        done_event.record(torch.cuda.current_stream() if stream is None else stream)
-    check(_lib.load().dsa_indexer_decode_host_async(*args, ctypes.c_void_p(done_event.cuda_event)))
+    _host_step("dsa_indexer_decode_host", q_host, w_host, k_new_host, dst_rows_host, cache,
+               _batch(seq_lens, q_lens, k_base), top_k, out_idx_host, out_score_host, q_scale_host, stream, done_event)
+
+
+def dsa_indexer_prefill_host(q_host, w_host, k_new_host, dst_rows_host, cache: IndexerKCache, seq_lens, top_k,
+                             out_idx_host, out_score_host, q_scale_host=None, q_lens=None, k_base=None, stream=None,
+                             done_event=None):
+    """One prefill step from HOST tensors in a single library call (dsa_indexer_prefill_host):
+    the same uploads, append and read-back as dsa_indexer_decode_host around the prefill's
+    scoring and selection (q_lens None: every key of a sequence has its query).  With
+    ``done_event`` the read-back of one step overlaps the next step's kernels."""
+    _host_step("dsa_indexer_prefill_host", q_host, w_host, k_new_host, dst_rows_host, cache,
+               _batch(seq_lens, q_lens, k_base), top_k, out_idx_host, out_score_host, q_scale_host, stream, done_event)
 
 
 def dsa_selftest_wait_expiry(limit_cycles=100000, stream=None):

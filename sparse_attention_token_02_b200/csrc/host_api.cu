@@ -905,17 +905,19 @@ static dsa_status_t ensure_step_streams(Ctx* c) {
   return DSA_OK;
 }
 
-// The host step.  Slot i % 2 holds step i's inputs and outputs:
+// The host step (decode, or prefill with the same copies).  Slot i % 2 holds step i's inputs
+// and outputs:
 //   copy_in : [wait computed(i-2)] H2D inputs            [record in_done(i)]
 //   stream  : [wait in_done(i), out_done(i-2)] append, quantise, decode   [record computed(i)]
 //   copy_out: [wait computed(i)] D2H outputs             [record out_done(i), done_event]
 // With join, `stream` then waits for out_done(i), so the host outputs are complete when the
 // stream is (the uploads of the next call still overlap this call's compute); without, the
 // caller waits on done_event.
-static dsa_status_t decode_host_step(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host, const void* k_new_host,
-                              dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host, int32_t n_new,
-                              const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host, float* out_score_host,
-                              void* stream_v, cudaEvent_t done_event, bool join) {
+static dsa_status_t host_step(bool prefill, const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                              const void* k_new_host, dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host,
+                              int32_t n_new, const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
+                              float* out_score_host, void* stream_v, cudaEvent_t done_event, bool join) {
+  const char* name = prefill ? "dsa_indexer_prefill_host" : "dsa_indexer_decode_host";
   g_last_error.clear();
   dsa_status_t st = check_cache(kc);
   if (st != DSA_OK) return st;
@@ -929,14 +931,14 @@ static dsa_status_t decode_host_step(const dsa_query_t* q, const dsa_kcache_t* k
   // bf16 queries against an FP8 cache are quantised on the device after the upload
   const bool quantise_q = q->dtype == DSA_BF16 && kc->dtype == DSA_FP8_E4M3;
   if (q->H_I <= 0 || q->d_I <= 0 || top_k <= 0) return fail(DSA_ERR_INVALID_ARG, "H_I, d_I and top_k must be positive");
-  if (batch->num_seqs < 0 || (batch->num_seqs > 0 && (!batch->seq_lens || !batch->q_lens)))
-    return fail(DSA_ERR_INVALID_ARG, "decode needs batch.seq_lens and batch.q_lens");
+  if (batch->num_seqs < 0 || (batch->num_seqs > 0 && (!batch->seq_lens || (!prefill && !batch->q_lens))))
+    return fail(DSA_ERR_INVALID_ARG, prefill ? "prefill needs batch.seq_lens" : "decode needs batch.seq_lens and batch.q_lens");
   int64_t T = 0;
-  for (int i = 0; i < batch->num_seqs; ++i) T += batch->q_lens[i];
+  for (int i = 0; i < batch->num_seqs; ++i) T += batch->q_lens ? batch->q_lens[i] : batch->seq_lens[i];
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   DSA_CUDA_TRY(cudaStreamIsCapturing(stream, &cap), "cudaStreamIsCapturing");
-  if (cap != cudaStreamCaptureStatusNone) return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_decode_host cannot be captured");
+  if (cap != cudaStreamCaptureStatusNone) return fail(DSA_ERR_UNSUPPORTED, "%s cannot be captured", name);
   Ctx* c = nullptr;
   if ((st = get_ctx(stream, &c)) != DSA_OK) return st;
   if ((st = ensure_step_streams(c)) != DSA_OK) return st;
@@ -995,8 +997,9 @@ static dsa_status_t decode_host_step(const dsa_query_t* q, const dsa_kcache_t* k
   }
   int32_t* oi = reinterpret_cast<int32_t*>(d + o_oi);
   float* os = reinterpret_cast<float*>(d + o_os);
-  if ((st = dsa_indexer_decode(&qd, kc, reinterpret_cast<const float*>(d + o_w), batch, top_k, oi, os, stream_v)) !=
-      DSA_OK)
+  const float* wd = reinterpret_cast<const float*>(d + o_w);
+  if ((st = prefill ? dsa_indexer_prefill(&qd, kc, wd, batch, top_k, oi, os, stream_v)
+                    : dsa_indexer_decode(&qd, kc, wd, batch, top_k, oi, os, stream_v)) != DSA_OK)
     return st;
   DSA_CUDA_TRY(cudaEventRecord(sl.computed, stream), "cudaEventRecord");
   DSA_CUDA_TRY(cudaStreamWaitEvent(c->copy_out, sl.computed, 0), "cudaStreamWaitEvent");
@@ -1015,8 +1018,8 @@ dsa_status_t dsa_indexer_decode_host(const dsa_query_t* q, const dsa_kcache_t* k
                                      const void* k_new_host, dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host,
                                      int32_t n_new, const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
                                      float* out_score_host, void* stream_v) {
-  return decode_host_step(q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
-                          out_score_host, stream_v, nullptr, true);
+  return host_step(false, q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
+                   out_score_host, stream_v, nullptr, true);
 }
 
 dsa_status_t dsa_indexer_decode_host_async(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
@@ -1028,8 +1031,29 @@ dsa_status_t dsa_indexer_decode_host_async(const dsa_query_t* q, const dsa_kcach
     g_last_error.clear();
     return fail(DSA_ERR_INVALID_ARG, "done_event is NULL");
   }
-  return decode_host_step(q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
-                          out_score_host, stream_v, static_cast<cudaEvent_t>(done_event), false);
+  return host_step(false, q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
+                   out_score_host, stream_v, static_cast<cudaEvent_t>(done_event), false);
+}
+
+dsa_status_t dsa_indexer_prefill_host(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                      const void* k_new_host, dsa_dtype_t k_new_dtype, const int64_t* dst_rows_host,
+                                      int32_t n_new, const dsa_batch_t* batch, int32_t top_k, int32_t* out_idx_host,
+                                      float* out_score_host, void* stream_v) {
+  return host_step(true, q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
+                   out_score_host, stream_v, nullptr, true);
+}
+
+dsa_status_t dsa_indexer_prefill_host_async(const dsa_query_t* q, const dsa_kcache_t* kc, const float* w_host,
+                                            const void* k_new_host, dsa_dtype_t k_new_dtype,
+                                            const int64_t* dst_rows_host, int32_t n_new, const dsa_batch_t* batch,
+                                            int32_t top_k, int32_t* out_idx_host, float* out_score_host,
+                                            void* stream_v, void* done_event) {
+  if (!done_event) {
+    g_last_error.clear();
+    return fail(DSA_ERR_INVALID_ARG, "done_event is NULL");
+  }
+  return host_step(true, q, kc, w_host, k_new_host, k_new_dtype, dst_rows_host, n_new, batch, top_k, out_idx_host,
+                   out_score_host, stream_v, static_cast<cudaEvent_t>(done_event), false);
 }
 
 // Over a cache of one key per m tokens the same kernels run with every query's causal limit

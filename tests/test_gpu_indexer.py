@@ -431,6 +431,51 @@ def test_decode_host_step_async_three_calls_in_flight(name):
     api.dsa_check_device_errors(s)
 
 
+@pytest.mark.parametrize("name", ["bf16", "fp8"])
+def test_prefill_host_step_matches_the_oracle_two_calls_and_three_in_flight(name):
+    # whole prefills from host memory: the keys appended (quantised for an FP8 cache), bf16
+    # queries uploaded (quantised on the device for an FP8 cache), the selection read back
+    base = W.prefill() if name == "bf16" else W.prefill8()
+    lens = (3000, 700)
+    wl = W.scaled(base, seq_lens=lens, q_lens=lens, seed=120)
+    up = Uploaded(wl)
+    k_h = torch.from_numpy(np.ascontiguousarray(np.concatenate(up.inp["k_bits"])).view(np.int16)).view(
+        torch.bfloat16).pin_memory()
+    rows_h = torch.arange(wl.total_k, dtype=torch.int64).pin_memory()
+    rows = list(range(0, wl.total_q, 37)) + [2047, 2048, 2999, 3000, wl.total_q - 1]
+    # two synchronous calls in a row
+    for call in range(2):
+        q_h = torch.from_numpy(np.ascontiguousarray(up.inp["q_bits"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        w_h = torch.from_numpy(up.inp["w"]).pin_memory()
+        oi_h = torch.full((wl.total_q, wl.top_k), 7, dtype=torch.int32).pin_memory()
+        os_h = torch.zeros((wl.total_q, wl.top_k), dtype=torch.float32).pin_memory()
+        s = torch.cuda.current_stream()
+        api.dsa_indexer_prefill_host(q_h, w_h, k_h, rows_h, up.cache, lens, wl.top_k, oi_h, os_h, k_base=up.k_base,
+                                     stream=s)
+        api.dsa_check_device_errors(s)
+        _check(up, oi_h.numpy(), os_h.numpy(), rows)
+    # three steps with different queries and weights in flight, each read back under its own event
+    s = torch.cuda.Stream()
+    steps = []
+    for call in range(3):
+        rng = np.random.default_rng(300 + call)
+        q_bits = W.f32_to_bf16_bits(rng.standard_normal(up.inp["q_bits"].shape).astype(np.float32))
+        w = W.softmax_rows(rng.standard_normal(up.inp["w"].shape).astype(np.float32))
+        q_h = torch.from_numpy(np.ascontiguousarray(q_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+        w_h = torch.from_numpy(w).pin_memory()
+        oi_h = torch.full((wl.total_q, wl.top_k), 7, dtype=torch.int32).pin_memory()
+        os_h = torch.zeros((wl.total_q, wl.top_k), dtype=torch.float32).pin_memory()
+        ev = torch.cuda.Event()
+        api.dsa_indexer_prefill_host(q_h, w_h, k_h, rows_h, up.cache, lens, wl.top_k, oi_h, os_h, k_base=up.k_base,
+                                     stream=s, done_event=ev)
+        steps.append((q_bits, w, q_h, w_h, oi_h, os_h, ev))
+    for q_bits, w, q_h, w_h, oi_h, os_h, ev in steps:
+        ev.synchronize()
+        ref = OracleInputs(wl, dict(up.inp, q_bits=q_bits, w=w))
+        _check(ref, oi_h.numpy(), os_h.numpy(), rows)
+    api.dsa_check_device_errors(s)
+
+
 def test_decode_host_step_rejects_bad_arguments():
     wl = W.scaled(W.decode(), seq_lens=(300,), q_lens=(1,))
     up = Uploaded(wl)
