@@ -889,8 +889,14 @@ __device__ bool row_sampled_select(const float* src, int n, uint32_t k, int32_t*
   // holds the k largest keys as soon as it has k elements.
   float4 cur[kRowEPT / 4];
   row_load(src, n, 0, cur);
+  // the histogram is idle during this pass: it stages each iteration's scores (kRowIter floats)
+  float* stage = reinterpret_cast<float*>(hist);
+  static_assert(kRowIter <= kRowBins0, "one iteration's scores fit the histogram buffer");
   auto gather = [&](auto tail, int base) {
     constexpr bool kTail = decltype(tail)::value;   // the last iteration: positions past n exist
+#pragma unroll
+    for (int v = 0; v < kRowEPT / 4; ++v)
+      *reinterpret_cast<float4*>(stage + (v * kRowThreads + tid) * 4) = cur[v];
     uint32_t sel = 0u;
 #pragma unroll
     for (int v = 0; v < kRowEPT / 4; ++v) {
@@ -911,24 +917,17 @@ __device__ bool row_sampled_select(const float* src, int n, uint32_t k, int32_t*
     uint32_t wbase = 0u;
     if (lane == 31 && incl) wbase = atomicAdd(ctr_a, incl);
     uint32_t slot = __shfl_sync(0xffffffffu, wbase, 31) + incl - mine;
-    // the selected keys, float4 by float4: a float4 with no selected key costs one test
-#pragma unroll
-    for (int v = 0; v < kRowEPT / 4; ++v) {
-      const uint32_t nib = (sel >> (4 * v)) & 0xFu;
-      if (nib) {
-        const float fv[4] = {cur[v].x, cur[v].y, cur[v].z, cur[v].w};
-        const int pos0 = base + (v * kRowThreads + tid) * 4;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if ((nib >> e) & 1u) {
-            if (slot < static_cast<uint32_t>(kRowCap)) {
-              cand_key[slot] = float_to_key(fv[e]);
-              cand_idx[slot] = pos0 + e;
-            }
-            ++slot;
-          }
-        }
+    // the selected keys, bit by bit: their values come back from this thread's own staged copy
+    // (written above, read by the same thread: no barrier needed)
+    while (sel) {
+      const int j = __ffs(sel) - 1;
+      sel &= sel - 1u;
+      if (slot < static_cast<uint32_t>(kRowCap)) {
+        const int local = ((j >> 2) * kRowThreads + tid) * 4 + (j & 3);
+        cand_key[slot] = float_to_key(stage[local]);
+        cand_idx[slot] = base + local;
       }
+      ++slot;
     }
   };
   int base = 0;
