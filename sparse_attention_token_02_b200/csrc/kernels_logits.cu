@@ -34,7 +34,10 @@ namespace dsa {
 
 namespace {
 
-constexpr int kScalePrefetch = 4;   // tiles of FP8 key scales in flight ahead of the epilogue
+#ifndef DSA_SCALE_PREFETCH
+#define DSA_SCALE_PREFETCH 4
+#endif
+constexpr int kScalePrefetch = DSA_SCALE_PREFETCH;   // tiles of FP8 key scales in flight ahead of the epilogue
 #ifndef DSA_TMEM_X64
 #define DSA_TMEM_X64 0                  // one 64-column TMEM load per query instead of two
 #endif

@@ -719,21 +719,27 @@ __global__ void __launch_bounds__(kStreamThreads) topk_stream_kernel(const TopkA
       ctr_b = 0u;
     }
     __syncthreads();
+    // slots per warp: one shared atomic per counter and warp instead of one per key (every
+    // thread calls f the same number of times, so the ballots see the whole warp)
+    const uint32_t lane_lt = (1u << (tid & 31)) - 1u;
     for_candidates<true, true, kStreamThreads, 8>(a.cand_key + off, a.cand_idx + off, bcount,
                                                    [&](uint32_t kk, int32_t ix, bool valid) {
-      if (!valid) return;
-      if (kk > sub_hi) {
-        const uint32_t t = atomicAdd(&ctr_a, 1u);
-        if (t < above1) {
-          oi[n_above_total + t] = ix;
-          os[n_above_total + t] = key_to_float(kk);
-        }
-      } else if (kk >= sub_lo) {
-        const uint32_t t = atomicAdd(&ctr_b, 1u);
-        if (t < static_cast<uint32_t>(kSubCap)) {
-          sub_key[t] = kk;
-          sub_idx[t] = ix;
-        }
+      const bool up = valid && kk > sub_hi;
+      const bool in = valid && !up && kk >= sub_lo;
+      const uint32_t bu = __ballot_sync(0xffffffffu, up), bi = __ballot_sync(0xffffffffu, in);
+      uint32_t tu = 0u, ti = 0u;
+      if ((tid & 31) == 0) {
+        if (bu) tu = atomicAdd(&ctr_a, static_cast<uint32_t>(__popc(bu)));
+        if (bi) ti = atomicAdd(&ctr_b, static_cast<uint32_t>(__popc(bi)));
+      }
+      tu = __shfl_sync(0xffffffffu, tu, 0) + __popc(bu & lane_lt);
+      ti = __shfl_sync(0xffffffffu, ti, 0) + __popc(bi & lane_lt);
+      if (up && tu < above1) {
+        oi[n_above_total + tu] = ix;
+        os[n_above_total + tu] = key_to_float(kk);
+      } else if (in && ti < static_cast<uint32_t>(kSubCap)) {
+        sub_key[ti] = kk;
+        sub_idx[ti] = ix;
       }
     });
     __syncthreads();
