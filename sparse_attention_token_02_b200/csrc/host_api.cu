@@ -778,8 +778,8 @@ dsa_status_t run_indexer(Mode mode, const dsa_query_t* q, const dsa_kcache_t* kc
     s.row_ctr = reinterpret_cast<uint32_t*>(wsb + wl.ctr);
     s.cand_key = reinterpret_cast<uint32_t*>(wsb + wl.cand_key);
     s.cand_idx = reinterpret_cast<int32_t*>(wsb + wl.cand_idx);
-    if (fp8) {
-      // the FP8 logits epilogue leaves the coarse histograms to a pass over the score rows
+    if (!logits_bins_rows(H, D, fp8, tpa, ng, prefill_items)) {
+      // this logits configuration leaves the coarse histograms to a pass over the score rows
       DSA_CUDA_TRY(launch_row_hist(s, stream), "row histogram launch");
       ++g_launches;
     }

@@ -105,6 +105,9 @@ struct LogitsLaunch {
 cudaError_t launch_logits(const LogitsLaunch& L, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q,
                           const LogitsArgs& a);
 bool logits_config_supported(int H, int D, bool fp8, int tpa, int ng, bool prefill);
+// Whether that configuration's epilogue counts every stored score in its row's coarse
+// histogram (the decode top-k then needs no pass of its own to build them).
+bool logits_bins_rows(int H, int D, bool fp8, int tpa, int ng, bool prefill);
 
 // Top-k over rows longer than top_k: one cluster of `cluster` CTAs per row,
 // `ept` keys per thread held in registers.

@@ -915,7 +915,7 @@ cudaError_t launch_cfg(const LogitsLaunch& L, const CUtensorMap& tk, const CUten
 #define DSA_D2F8_NE 8
 #endif
 #ifndef DSA_D2F8_STAGES
-#define DSA_D2F8_STAGES 10
+#define DSA_D2F8_STAGES 8
 #endif
 #ifndef DSA_D2F8_EG
 #define DSA_D2F8_EG 1
@@ -979,6 +979,16 @@ cudaError_t launch_logits(const LogitsLaunch& L, const CUtensorMap& tk, const CU
   if (L.H == 4 && L.D == 64 && !L.fp8 && L.tpa == 64 && L.ng == 1)
     return launch_cfg<CfgPrefillSmallH>(L, tk, tq, a);
   return cudaErrorInvalidValue;
+}
+
+bool logits_bins_rows(int H, int D, bool fp8, int tpa, int ng, bool prefill) {
+  if (H != 64 || D != 128 || prefill || ng != 1) return false;
+  switch (tpa) {
+    case 1: return fp8 ? CfgDecode1Fp8::HIST : CfgDecode1Bf16::HIST;
+    case 2: return fp8 ? CfgDecode2Fp8::HIST : CfgDecode2Bf16::HIST;
+    case 4: return fp8 ? CfgDecode4Fp8::HIST : CfgDecode4Bf16::HIST;
+    default: return false;
+  }
 }
 
 int logits_queries_per_item(int H, int D, bool prefill, int max_q_len) {

@@ -54,7 +54,9 @@ def test_append_bf16_copy_and_f32_rounding():
     api.dsa_check_device_errors()
 
 
-@pytest.mark.parametrize("row_len", [128, 8192])
+# 128: a key row (one warp each); 1040, 8192, 9008: one CTA per row with 1, 4 and 8 chunks of 8 values
+# per thread, the first and last ragged; 16400: past the CTA kernel's register capacity (warp loop)
+@pytest.mark.parametrize("row_len", [128, 1040, 8192, 9008, 16400])
 def test_quantize_rows_fp8_bit_exact_against_oracle_codec(row_len):
     rng = np.random.default_rng(row_len)
     x = (rng.standard_normal((257, row_len)) * rng.uniform(1e-3, 50, (257, 1))).astype(np.float32)
