@@ -159,12 +159,29 @@ __device__ __forceinline__ void for_candidates(const uint32_t* ck, const int32_t
   }
 }
 
+// Sorts one key per lane of a warp in descending order across the lanes (bitonic network).
+__device__ __forceinline__ uint32_t warp_sort_desc(uint32_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool asc = (lane & k) == 0, low = (lane & j) == 0;
+      v = low == asc ? max(v, o) : min(v, o);
+    }
+  }
+  return v;
+}
+
 // One CTA, all its threads: the m gathered keys (in this CTA's shared memory, or with
 // kGlobalCand in global memory, read through the L2 since other CTAs wrote them) are
 // n_up keys above hi, all selected, and m - n_up keys in [lo, hi] of which the `need`
 // largest are selected; all n_up + need go to slots [base, base + n_up + need) of the row.
-// Exact: CTA-local histogram levels narrow [lo, hi] by >= 2^10 per level; keys above the
-// final interval are taken, then `need` of its keys (a single tied value if not resolved).
+// Exact: CTA-local histogram levels narrow [lo, hi] by >= 2^10 per level; once the interval
+// holds at most 32 keys one warp sorts them and the need-th largest value v becomes the
+// interval [v, v] (the keys above v join the selected ones); keys above the final interval are
+// taken, then `need` of its keys (a single tied value if not resolved).
 // Returns false if the counts turn out inconsistent (nothing is written past the row).
 template <bool kGlobalCand, int NT>
 __device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, uint32_t m, uint32_t n_up,
@@ -179,8 +196,42 @@ __device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, 
   ls.hi = hi;
   ls.need = need;
   ls.done = need == m - n_up ? 1u : 0u;
-  for (int level = 0; level < 4 && !ls.done; ++level) {
+  uint32_t cnt = m - n_up;                    // keys inside [lo, hi]
+  for (int level = 0; level < 5 && !ls.done; ++level) {
     if (ls.lo == ls.hi) { ls.done = 2; break; }
+    if (cnt <= 32u) {
+      // few keys left: gather them (key, position) into the histogram's first 64 words, sort
+      // them in one warp, and keep the need-th largest value as a one-value interval
+      if (tid == 0) *ctr_a = 0u;
+      __syncthreads();
+      for_candidates<kGlobalCand, true, NT, CPT>(cand_key, cand_idx, m, [&](uint32_t kk, int32_t ix, bool valid) {
+        if (valid && kk >= ls.lo && kk <= ls.hi) {
+          const uint32_t slot = atomicAdd(ctr_a, 1u);
+          if (slot < 32u) {
+            hist[slot] = kk;
+            hist[32 + slot] = static_cast<uint32_t>(ix);
+          }
+        }
+      });
+      __syncthreads();
+      if (*ctr_a != cnt) return false;        // inconsistent counts (uniform: read after the barrier)
+      if (tid < 32) {
+        const uint32_t v = warp_sort_desc(tid < static_cast<int>(cnt) ? hist[tid] : 0u);
+        const uint32_t vk = __shfl_sync(0xffffffffu, v, static_cast<int>(ls.need) - 1);
+        const uint32_t gt = __popc(__ballot_sync(0xffffffffu, v > vk));
+        if (tid == 0) {
+          *lvl_bin = vk;
+          *lvl_above = gt;
+        }
+      }
+      __syncthreads();
+      ls.lo = *lvl_bin;
+      ls.hi = ls.lo;
+      ls.need -= *lvl_above;
+      ls.done = 2;
+      __syncthreads();                        // lvl_* and ctr_a are reused below
+      break;
+    }
     const int bits = 32 - __clz(ls.hi - ls.lo);
     const int shift = bits > 11 ? bits - 11 : 0;
     for (int b = tid; b < kBins; b += NT) hist[b] = 0u;
@@ -202,6 +253,7 @@ __device__ bool rank0_select(const uint32_t* cand_key, const int32_t* cand_idx, 
     ns.hi = (ls.hi - ns.lo) > width_m1 ? ns.lo + width_m1 : ls.hi;
     ns.need = ls.need - *lvl_above;
     ns.done = *lvl_cnt == ns.need ? 1u : 0u;
+    cnt = *lvl_cnt;
     ls = ns;
     __syncthreads();
   }
