@@ -94,7 +94,7 @@ def test_decode_bf16_cluster_rows_of_16k_to_32k_keys(q_len):
 
 def test_decode_bf16_rows_beyond_32k_keys_stream():
     # one row longer than a 4-CTA cluster holds sends every row of the batch to the streaming top-k
-    lens = (40000, 33000, 5000, 2049, 32768)
+    lens = (40000, 33000, 5000, 2049, 32768, 8192, 8193)
     wl = W.scaled(W.decode(), seq_lens=lens, q_lens=(2,) * len(lens), seed=64)
     up = Uploaded(wl)
     idx, sc = run_indexer(up, decode=True)
@@ -115,8 +115,9 @@ def test_prefill_rows_beyond_4096_keys_take_the_sampled_threshold(name):
 
 
 def test_ragged_decode_fp8_longest_and_shortest_rows():
-    # FP8 decode: the row-histogram pass and the streaming top-k over 4096 .. 131072 keys
-    lens = (131072, 4096, 70001, 4097)
+    # FP8 decode: the row-histogram pass and the streaming top-k over 4096 .. 131072 keys; rows at
+    # the chunk boundaries (one, two and three chunks of 4096 keys, and five)
+    lens = (131072, 4096, 70001, 4097, 8192, 8193, 16385)
     wl = W.scaled(W.decode8(), seq_lens=lens, q_lens=(2,) * len(lens), seed=72)
     up = Uploaded(wl)
     idx, sc = run_indexer(up, decode=True)
