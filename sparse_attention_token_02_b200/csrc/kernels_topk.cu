@@ -341,6 +341,10 @@ topk_kernel(const TopkArgs a) {
     lvl_cnt = 0u;
   }
   __syncthreads();
+  // rank 0's counters are zeroed before any CTA of the cluster touches them remotely: arrive
+  // now, wait just before the first access to another CTA's shared memory (by then every CTA
+  // has long arrived, so the wait costs nothing)
+  cluster_arrive();
   grid_dependency_wait();                     // the scores come from the previous kernel
 
   // ---- the row's coarse histogram, when the logits epilogue built one (decode)
@@ -376,8 +380,10 @@ topk_kernel(const TopkArgs a) {
     __syncthreads();
     bin_lo = lvl_bin << kHistShift;
     bin_hi = bin_lo | ((1u << kHistShift) - 1u);
+    cluster_wait();
   } else {
     // ---- data-driven first level: bins spread over the row's key range
+    cluster_wait();
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));

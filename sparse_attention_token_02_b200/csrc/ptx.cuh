@@ -101,6 +101,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Split cluster barrier: arrive (release: this thread's shared-memory writes so far become
+// visible to the cluster) and wait (acquire: every CTA of the cluster has arrived).  Every thread
+// of every CTA in the cluster executes both, in this order, before its next cluster barrier.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
