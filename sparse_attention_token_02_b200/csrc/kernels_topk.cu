@@ -298,6 +298,7 @@ template <int EPT>
 __global__ void __launch_bounds__(kThreads, EPT <= 8 ? 2 : 1)
 topk_kernel(const TopkArgs a) {
   static_assert(EPT % 4 == 0, "EPT is a multiple of 4");
+  static_assert(EPT * kThreads < 65536, "per-CTA counts are packed in 16 bits");
   extern __shared__ __align__(16) uint32_t dsm[];
   uint32_t* hist = dsm;                                             // kBins
   uint32_t* cand_key = dsm + kBins;                                 // kCandCap
@@ -457,21 +458,21 @@ topk_kernel(const TopkArgs a) {
 
   if (bcount <= static_cast<uint32_t>(kCandCap)) {
     // ---- write the keys above the bin, gather the bin's keys into rank 0
+    // both counts in one scan (each < 2^16 per CTA); the two slot atomics on rank 0 from two
+    // warps, so that their round trips overlap
     uint32_t n_up = 0, n_in = 0;
 #pragma unroll
     for (int e = 0; e < EPT; ++e) {
       n_up += key[e] > bin_hi;
       n_in += key[e] >= bin_lo && key[e] <= bin_hi;
     }
-    uint32_t tot_up, tot_in;
-    const uint32_t pre_up = block_exclusive_scan(n_up, warp_sums, tot_up);
-    const uint32_t pre_in = block_exclusive_scan(n_in, warp_sums, tot_in);
-    if (tid == 0) {
-      base_above = tot_up ? atomicAdd(cnt_above0, tot_up) : 0u;
-      base_cand = tot_in ? atomicAdd(cnt_cand0, tot_in) : 0u;
-    }
+    uint32_t tot;
+    const uint32_t pre = block_exclusive_scan((n_up << 16) | n_in, warp_sums, tot);
+    const uint32_t tot_up = tot >> 16, tot_in = tot & 0xFFFFu;
+    if (tid == 0) base_above = tot_up ? atomicAdd(cnt_above0, tot_up) : 0u;
+    if (tid == 32) base_cand = tot_in ? atomicAdd(cnt_cand0, tot_in) : 0u;
     __syncthreads();
-    uint32_t iu = base_above + pre_up, ic = base_cand + pre_in;
+    uint32_t iu = base_above + (pre >> 16), ic = base_cand + (pre & 0xFFFFu);
 #pragma unroll
     for (int v = 0; v < EPT / 4; ++v) {
 #pragma unroll
